@@ -1,0 +1,194 @@
+"""CPU oracle for the tree speculative-decoding verification step.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference arm are the only callers.  The product
+package never imports this module, and this module never imports the product
+package.  The arithmetic lives in ``oracle.c`` (plain C, no CUDA headers); this
+file only compiles it with gcc and marshals numpy arrays through ctypes.
+
+Sources: "EAGLE-Pangu: Accelerator-Safe Tree Speculative Decoding on Ascend
+NPUs" (methodology A-C, results) and "Batch Speculative Decoding Done Right"
+(methodology: synchronization invariants, EQSPEC).  Each C function names the
+passage it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+BAD_PARENT = 1
+TOO_DEEP = 2
+BAD_GEOMETRY = 8
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        _lib.oracle_tree_build_mask.argtypes = [P, i32, i32, i32, P, P, P]
+        _lib.oracle_tree_attention_rows.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, P, i64, P]
+        _lib.oracle_tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, P]
+        _lib.oracle_argmax_rows.argtypes = [P, i64, i32, P]
+        _lib.oracle_tree_accept.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P]
+        _lib.oracle_kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P]
+        for f in (
+            _lib.oracle_tree_build_mask,
+            _lib.oracle_tree_attention_rows,
+            _lib.oracle_tree_attention,
+            _lib.oracle_argmax_rows,
+            _lib.oracle_tree_accept,
+            _lib.oracle_kv_commit_realign,
+        ):
+            f.restype = ctypes.c_int
+    return _lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a
+
+
+def _p(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _bits16(a: np.ndarray) -> np.ndarray:
+    """bf16 payload as uint16 bits (accepts uint16 bits or torch-exported int16 views)."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return a
+    if a.dtype == np.int16:
+        return a.view(np.uint16)
+    raise TypeError("bf16 tensors must be passed as uint16 bit patterns")
+
+
+def tree_build_mask(parent: np.ndarray, max_depth: int):
+    """parent int32 [B][M+1] -> (anc_mask uint32 [B][M+1][W], depth int32 [B][M+1], status int32 [B])."""
+    parent = _c(parent, np.int32)
+    B, n = parent.shape
+    M = n - 1
+    W = (n + 31) // 32
+    anc = np.zeros((B, n, W), np.uint32)
+    depth = np.zeros((B, n), np.int32)
+    status = np.zeros((B,), np.int32)
+    rc = lib().oracle_tree_build_mask(_p(parent), B, M, max_depth, _p(anc), _p(depth), _p(status))
+    if rc:
+        raise ValueError("oracle_tree_build_mask rc=%d" % rc)
+    return anc, depth, status
+
+
+def tree_attention(q, k, v, kv_start, kv_len, parent, status, Hkv: int, scale: float | None = None):
+    """q bf16-bits [B][M+1][Hq][D]; k, v bf16-bits [B][Hkv][S_cap][D] -> float64 [B][M+1][Hq][D]."""
+    q, k, v = _bits16(q), _bits16(k), _bits16(v)
+    B, n, Hq, D = q.shape
+    S_cap = k.shape[2]
+    assert k.shape == (B, Hkv, S_cap, D) and v.shape == k.shape
+    ks, kl = _c(kv_start, np.int32), _c(kv_len, np.int32)
+    par, st = _c(parent, np.int32), _c(status, np.int32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((B, n, Hq, D), np.float64)
+    rc = lib().oracle_tree_attention(
+        _p(q), _p(k), _p(v), S_cap, _p(ks), _p(kl), _p(par), _p(st), B, n - 1, Hq, Hkv, D, scale, _p(out)
+    )
+    if rc:
+        raise ValueError("oracle_tree_attention rc=%d" % rc)
+    return out
+
+
+def tree_attention_rows(q, k, v, kv_start, kv_len, parent, status, Hkv: int, sel, scale: float | None = None):
+    """Only the rows listed in sel ([n][3] of (b, u, q_head)) -> float64 [n][D]."""
+    q, k, v = _bits16(q), _bits16(k), _bits16(v)
+    B, n, Hq, D = q.shape
+    S_cap = k.shape[2]
+    ks, kl = _c(kv_start, np.int32), _c(kv_len, np.int32)
+    par, st = _c(parent, np.int32), _c(status, np.int32)
+    sel = _c(sel, np.int32).reshape(-1, 3)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.zeros((sel.shape[0], D), np.float64)
+    rc = lib().oracle_tree_attention_rows(
+        _p(q), _p(k), _p(v), S_cap, _p(ks), _p(kl), _p(par), _p(st), B, n - 1, Hq, Hkv, D, scale,
+        _p(sel), sel.shape[0], _p(out),
+    )
+    if rc:
+        raise ValueError("oracle_tree_attention_rows rc=%d" % rc)
+    return out
+
+
+def argmax_rows(logits):
+    logits = _c(logits, np.float32)
+    V = logits.shape[-1]
+    rows = logits.size // V
+    out = np.zeros((rows,), np.int32)
+    lib().oracle_argmax_rows(_p(logits), rows, V, _p(out))
+    return out.reshape(logits.shape[:-1])
+
+
+def tree_accept(logits, draft, parent, status, max_depth: int):
+    """-> (argmax [B][M+1], accept_len [B], path [B][max_depth+1], bonus [B])."""
+    logits = _c(logits, np.float32)
+    B, n, V = logits.shape
+    dr, par, st = _c(draft, np.int32), _c(parent, np.int32), _c(status, np.int32)
+    am = np.zeros((B, n), np.int32)
+    al = np.zeros((B,), np.int32)
+    path = np.zeros((B, max_depth + 1), np.int32)
+    bonus = np.zeros((B,), np.int32)
+    rc = lib().oracle_tree_accept(
+        _p(logits), _p(dr), _p(par), _p(st), B, n - 1, V, max_depth, _p(am), _p(al), _p(path), _p(bonus)
+    )
+    if rc:
+        raise AssertionError("oracle_tree_accept: recurrence and brute force disagree (rc=%d)" % rc)
+    return am, al, path, bonus
+
+
+def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_depth: int,
+                      kv_start, kv_len, realign: int, with_mask: bool = True):
+    """In place on the uint16 arrays in k_layers / v_layers (each [B][Hkv][S_cap][D]).
+
+    Returns (kv_start', kv_len', max_len', attn_mask or None, pos_ids or None)."""
+    L = len(k_layers)
+    assert L == len(v_layers) and L >= 1
+    B, Hkv, S_cap, D = k_layers[0].shape
+    for a in list(k_layers) + list(v_layers):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous and a.shape == (B, Hkv, S_cap, D)
+    kp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in k_layers])
+    vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_layers])
+    ks = _c(kv_start, np.int32).copy()
+    kl = _c(kv_len, np.int32).copy()
+    pth, al, st = _c(path, np.int32), _c(accept_len, np.int32), _c(status, np.int32)
+    ml = np.zeros((1,), np.int32)
+    am = np.zeros((B, S_cap), np.uint8) if with_mask else None
+    pos = np.zeros((B, S_cap), np.int32) if with_mask else None
+    rc = lib().oracle_kv_commit_realign(
+        ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), L, B, Hkv, D, S_cap, M,
+        _p(pth), _p(al), _p(st), max_depth, _p(ks), _p(kl), _p(ml), int(realign),
+        _p(am) if with_mask else None, _p(pos) if with_mask else None,
+    )
+    if rc:
+        raise ValueError("oracle_kv_commit_realign rc=%d" % rc)
+    return ks, kl, int(ml[0]), am, pos
