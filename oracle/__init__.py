@@ -167,10 +167,11 @@ def tree_accept(logits, draft, parent, status, max_depth: int):
 
 
 def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_depth: int,
-                      kv_start, kv_len, realign: int, with_mask: bool = True):
+                      kv_start, kv_len, realign: int, with_mask: bool = True, with_status: bool = False):
     """In place on the uint16 arrays in k_layers / v_layers (each [B][Hkv][S_cap][D]).
 
-    Returns (kv_start', kv_len', max_len', attn_mask or None, pos_ids or None)."""
+    Returns (kv_start', kv_len', max_len', attn_mask or None, pos_ids or None);
+    with_status=True appends status' (input status with TV_SEQ_BAD_GEOMETRY OR-ed in)."""
     L = len(k_layers)
     assert L == len(v_layers) and L >= 1
     B, Hkv, S_cap, D = k_layers[0].shape
@@ -180,7 +181,8 @@ def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_
     vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_layers])
     ks = _c(kv_start, np.int32).copy()
     kl = _c(kv_len, np.int32).copy()
-    pth, al, st = _c(path, np.int32), _c(accept_len, np.int32), _c(status, np.int32)
+    pth, al = _c(path, np.int32), _c(accept_len, np.int32)
+    st = _c(status, np.int32).copy()
     ml = np.zeros((1,), np.int32)
     am = np.zeros((B, S_cap), np.uint8) if with_mask else None
     pos = np.zeros((B, S_cap), np.int32) if with_mask else None
@@ -191,4 +193,6 @@ def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_
     )
     if rc:
         raise ValueError("oracle_kv_commit_realign rc=%d" % rc)
+    if with_status:
+        return ks, kl, int(ml[0]), am, pos, st
     return ks, kl, int(ml[0]), am, pos

@@ -311,15 +311,16 @@ int oracle_tree_accept(const float* logits, const int32_t* draft, const int32_t*
  * the batch maximum for every b, (ii) position IDs contiguous from 0 over the
  * attended (mask = 1) positions.
  * Reading adopted: the committed rows are the root row plus the accepted nodes
- * (a+1 rows, root first); a sequence with status != 0 commits nothing; a
- * sequence with an out-of-range cache geometry is left untouched.
+ * (a+1 rows, root first); a sequence with status != 0, or whose path points
+ * outside the tree, commits nothing; a sequence with an out-of-range cache
+ * geometry is left untouched and flagged in status.
  * k_layers / v_layers are host arrays of L host pointers to [B][Hkv][S_cap][D].
  * realign = 0: per-sequence lengths (content stays at kv_start).
  * realign = 1: left-padded; content is repadded to end at the new batch maximum.
  * ------------------------------------------------------------------------- */
 int oracle_kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers, int L, int B,
                              int Hkv, int D, int64_t S_cap, int M, const int32_t* path,
-                             const int32_t* accept_len, const int32_t* status, int max_depth,
+                             const int32_t* accept_len, int32_t* status, int max_depth,
                              int32_t* kv_start, int32_t* kv_len, int32_t* max_len, int realign,
                              uint8_t* attn_mask, int32_t* pos_ids) {
   int32_t* nb = (int32_t*)calloc((size_t)(B > 0 ? B : 1), sizeof(int32_t));
@@ -330,6 +331,11 @@ int oracle_kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layer
     good[b] = geometry_ok(kv_start[b], kv_len[b], M, S_cap);
     int a = accept_len[b];
     nb[b] = (good[b] && status[b] == 0 && a >= 0 && a <= max_depth && a <= M) ? a + 1 : 0;
+    /* a path row outside [0, M] would gather outside the tree: commit nothing */
+    for (int j = 0; j < nb[b]; ++j) {
+      int r = path[(int64_t)b * (max_depth + 1) + j];
+      if (r < 0 || r > M) nb[b] = 0;
+    }
     if (good[b]) {
       int64_t nl = (int64_t)kv_len[b] + nb[b];
       int64_t end = realign ? nl : (int64_t)kv_start[b] + nl;
@@ -369,6 +375,8 @@ int oracle_kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layer
     if (good[b]) {
       kv_len[b] += nb[b];
       kv_start[b] = new_start[b];
+    } else {
+      status[b] |= OR_BAD_GEOMETRY;
     }
     if (attn_mask || pos_ids)
       for (int64_t t = 0; t < S_cap; ++t) {

@@ -229,3 +229,21 @@ def test_bad_geometry_left_untouched(orc):
     np.testing.assert_array_equal(k[1], before[1])
     assert ks2[1] == 0 and kl2[1] == 14 and not mask[1].any()
     assert ks2[0] == 0 and kl2[0] == 7 and ml == 7
+
+
+def test_out_of_tree_path_commits_nothing(orc):
+    B, Hkv, D, M, md = 2, 1, 4, 3, 3
+    S_cap = 20
+    k = _ids_cache(B, Hkv, S_cap, D)
+    v = k.copy()
+    before = k.copy()
+    ks = np.array([0, 0], np.int32)
+    kl = np.array([5, 6], np.int32)
+    path = np.array([[0, 1, 9, 0], [0, 2, 0, 0]], np.int32)  # row 9 does not exist (M = 3)
+    al = np.array([2, 1], np.int32)
+    ks2, kl2, ml, _, _, st = orc.kv_commit_realign(
+        [k], [v], M, path, al, np.zeros(B, np.int32), md, ks, kl, realign=0, with_status=True
+    )
+    assert kl2.tolist() == [5, 8] and ml == 8 and st.tolist() == [0, 0]
+    np.testing.assert_array_equal(k[0], before[0])
+    np.testing.assert_array_equal(k[1, :, 6 + 1], before[1, :, 6 + 2])
