@@ -1,0 +1,181 @@
+/*
+ * treeverify.h -- C ABI of the teacher-side verification step of tree
+ * speculative decoding, for NVIDIA B200 (sm_100a).
+ *
+ * The step, as the pages state it:
+ *   "EAGLE-Pangu: Accelerator-Safe Tree Speculative Decoding on Ascend NPUs"
+ *     methodology B  sentinel-free tree tensors: a dummy root at row 0, every
+ *                    parent pointer in [0, M], invariants (in range, acyclic)
+ *                    checked before the fused kernels run;
+ *     methodology C  one batched teacher pass over all speculative tokens with a
+ *                    tree mask: node k attends node j only if j is an ancestor
+ *                    of k (itself included);
+ *     methodology A  path-index commit: the new cache segment is reordered by
+ *                    the accepted path ("fast reorder");
+ *     results        accepted length per verification step (greedy agreement).
+ *   "Batch Speculative Decoding Done Right"
+ *     methodology    EQSPEC unpad-append-repad, keeping rectangular alignment
+ *                    (pad + length = batch maximum) and position IDs contiguous
+ *                    from 0 over the attended positions.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  Nothing is
+ *     allocated, nothing is kept between calls.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ *     stream) and never synchronises.  The return value reports only argument
+ *     errors and launch errors, detected synchronously on the host.
+ *   - Data-dependent errors are reported on the device, per sequence, in the
+ *     int32 `status[B]` array (bit flags below).  A sequence with status != 0
+ *     gets zero attention rows, accept_len = -1 with a zero path, and commits
+ *     nothing (in left-padded mode it is still shifted to keep the batch
+ *     rectangular).
+ *   - Indices are int32 and never negative (except accept_len = -1); padding of
+ *     index arrays uses 0, the dummy root, so any gather stays in bounds.
+ *   - Trees have M+1 rows: row 0 is the dummy root (the last emitted token, not
+ *     yet in the cache), rows 1..M are draft nodes, parent[0] = 0 and
+ *     0 <= parent[i] < i.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - KV cache of one layer: [B][Hkv][S_cap][D] bf16.  Sequence b's committed
+ *     prefix is columns [kv_start[b], kv_start[b] + kv_len[b]); the caller has
+ *     written the M+1 tree rows of the current step right behind it, at columns
+ *     kv_start[b] + kv_len[b] + r, r = 0..M.  A sequence whose geometry breaks
+ *     0 <= kv_start, 0 <= kv_len, kv_start + kv_len + M + 1 <= S_cap is flagged
+ *     TV_SEQ_BAD_GEOMETRY and skipped.
+ */
+#ifndef TREEVERIFY_H
+#define TREEVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st* tv_stream_t;
+
+typedef enum {
+  TV_OK = 0,
+  TV_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer, bad combination */
+  TV_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement (e.g. D not 64/128) */
+  TV_ERR_CUDA = 3         /* a CUDA runtime call or launch failed; see tv_last_cuda_error() */
+} tv_status;
+
+/* per-sequence device status bits */
+#define TV_SEQ_BAD_PARENT 1   /* parent[0] != 0, or parent[i] outside [0, i) */
+#define TV_SEQ_TOO_DEEP 2     /* some node deeper than max_depth */
+#define TV_SEQ_TIMEOUT 4      /* a bounded device wait gave up (the sequence's outputs are void) */
+#define TV_SEQ_BAD_GEOMETRY 8 /* kv_start / kv_len / S_cap inconsistent with M+1 tree rows */
+
+/* Largest tree the kernels take: M + 1 <= TV_MAX_TREE_ROWS. */
+#define TV_MAX_TREE_ROWS 256
+
+/*
+ * tree_build_mask -- validate sentinel-free parent arrays and expand them into
+ * ancestor bitmasks.  [EAGLE-Pangu, methodology B (dummy-root indexing,
+ * ancestor tables, invariant checks) and C (tree attention mask).]
+ *
+ *   parent    int32 [B][M+1]   in
+ *   anc_mask  uint32 [B][M+1][W], W = ceil((M+1)/32)   out: bit r of row u is
+ *             set iff row r lies on the root..u path, u included
+ *   depth     int32 [B][M+1]   out: edges from the root (root = 0)
+ *   status    int32 [B]        out: 0, or TV_SEQ_BAD_PARENT / TV_SEQ_TOO_DEEP;
+ *             a flagged sequence gets all-zero mask and depth rows
+ *   B >= 0, 0 <= M < TV_MAX_TREE_ROWS, max_depth >= 0.
+ */
+tv_status tree_build_mask(const int32_t* parent, int B, int M, int max_depth, uint32_t* anc_mask,
+                          int32_t* depth, int32_t* status, tv_stream_t stream);
+
+/*
+ * tree_attention -- tree-masked GQA attention of the M+1 tree queries of every
+ * sequence over its committed prefix plus its tree rows.  [EAGLE-Pangu,
+ * methodology C: one batched pass over all speculative tokens; node u attends
+ * the whole prefix, and inside the tree only rows whose bit is set in
+ * anc_mask[b][u].]
+ *
+ *   q         bf16 [B][M+1][Hq][D]       in (post-RoPE)
+ *   k, v      bf16 [B][Hkv][S_cap][D]    in (one layer); 16-byte aligned
+ *   kv_start, kv_len  int32 [B]          in
+ *   anc_mask  uint32 [B][M+1][W]         in (from tree_build_mask)
+ *   status    int32 [B]                  in/out: sequences with status != 0 are
+ *             skipped (zero output); bad geometry / wait timeouts are OR-ed in
+ *   out       bf16 [B][M+1][Hq][D]       out: softmax(q k^T * scale) v over the
+ *             allowed keys, fp32 accumulation
+ *   D in {64, 128}; Hq % Hkv == 0 (q head h reads kv head h / (Hq/Hkv));
+ *   scale > 0 (normally 1/sqrt(D)).
+ * Contract: the K/V rows inside each sequence's key range hold finite values.
+ */
+tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                         const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
+                         int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
+                         uint16_t* out, tv_stream_t stream);
+
+/*
+ * tree_accept -- per-node greedy argmax of the teacher logits fused with
+ * longest accepted path selection.  [EAGLE-Pangu, results: accepted length per
+ * verification step.]  Node i is accepted iff its parent is accepted and
+ * draft[i] == argmax[parent[i]]; the root is always accepted.  The committed
+ * endpoint e is the deepest accepted node, lowest row index on ties.
+ *
+ *   logits     fp32 [B][M+1][V]   in (row u predicts the children of node u)
+ *   draft      int32 [B][M+1]     in (draft token of node i; row 0 ignored)
+ *   parent, depth  int32 [B][M+1], anc_mask uint32 [B][M+1][W]   in
+ *   status     int32 [B]          in/out: non-zero -> sequence rejected
+ *   argmax     int32 [B][M+1]     out: first index of the row maximum
+ *   accept_len int32 [B]          out: depth of e (accepted draft tokens), -1 if rejected
+ *   path       int32 [B][max_depth+1]  out: path[j] = row of depth j on root..e, 0-padded
+ *   bonus      int32 [B]          out: argmax[e] (the teacher's next token), 0 if rejected
+ *   V >= 1; max_depth must be the value given to tree_build_mask.
+ * Contract: logits are finite (NaN ordering is unspecified).
+ */
+tv_status tree_accept(const float* logits, const int32_t* draft, const int32_t* parent,
+                      const int32_t* depth, const uint32_t* anc_mask, int32_t* status, int B, int M,
+                      int V, int max_depth, int32_t* argmax, int32_t* accept_len, int32_t* path,
+                      int32_t* bonus, tv_stream_t stream);
+
+/*
+ * kv_commit_realign -- commit the accepted path into the KV cache of every
+ * layer and, in left-padded mode, repad the batch.  [EAGLE-Pangu, methodology A:
+ * path-index commit; Batch Speculative Decoding Done Right, methodology:
+ * EQSPEC unpad-append-repad and its two invariants.]
+ *
+ * For sequence b with n_b = accept_len[b] + 1 committed rows (0 if rejected):
+ *   new content = old content ++ { tail row path[b][j] : j < n_b }, where the
+ *   tail is the M+1 tree rows behind the content; kv_len[b] += n_b.
+ *   realign = 0  per-sequence lengths: content stays at kv_start[b].
+ *   realign = 1  left-padded: with Lmax' = max_b kv_len'[b], content moves to
+ *                [Lmax' - kv_len'[b], Lmax'); kv_start'[b] = Lmax' - kv_len'[b].
+ * All sources are read before they are overwritten (moves are in place).
+ *
+ *   k_layers, v_layers  DEVICE arrays of L device pointers, each to a
+ *             bf16 [B][Hkv][S_cap][D] layer (16-byte aligned)
+ *   path, accept_len, status   in (from tree_accept); status gains
+ *             TV_SEQ_BAD_GEOMETRY for skipped sequences
+ *   kv_start, kv_len  int32 [B]   in/out
+ *   max_len   int32 [1]           out: max_b kv_start'[b] + kv_len'[b] over
+ *             sequences with a valid geometry (Lmax' in left-padded mode)
+ *   attn_mask uint8 [B][S_cap], pos_ids int32 [B][S_cap]   out, may be NULL:
+ *             mask = 1 on the new content columns, pos = column - kv_start',
+ *             0 elsewhere
+ */
+tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers, int L, int B,
+                            int Hkv, int D, int64_t S_cap, int M, const int32_t* path,
+                            const int32_t* accept_len, int32_t* status, int max_depth,
+                            int32_t* kv_start, int32_t* kv_len, int32_t* max_len, int realign,
+                            uint8_t* attn_mask, int32_t* pos_ids, tv_stream_t stream);
+
+/* Human-readable name of a tv_status. */
+const char* tv_status_string(tv_status s);
+
+/* The cudaError_t of the most recent TV_ERR_CUDA returned on this thread (0 if none). */
+int tv_last_cuda_error(void);
+
+/* ABI version (major * 100 + minor). */
+int tv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TREEVERIFY_H */

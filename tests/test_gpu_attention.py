@@ -1,0 +1,147 @@
+"""GPU parity of tree_attention against the oracle.
+
+Tolerance (bf16 inputs, fp32 accumulation, bf16 output): |gpu - ref| <= 1e-2 +
+2e-2 |ref| elementwise.  Small and mid-size workloads are compared on every
+output row; the two largest are compared on a seeded sample of rows (plus every
+row of sequence 0) in the launch configuration the benchmark uses.  Also: the
+leak test (non-ancestor V rows = 1e4), invalid sequences give zero rows, GQA
+groups, head dims 64/128, empty prefixes, single-node trees and the largest
+tree the kernels take.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import dev, gpu_attention, gpu_mask, i32
+from helpers import assert_attn_close
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(orc, q, k, v, parent, kv_start, kv_len, max_depth=1000, status_override=None, sel=None):
+    par, anc, depth, status = gpu_mask(parent, max_depth)
+    if status_override is not None:
+        status.copy_(i32(status_override))
+    st_h = status.cpu().numpy()
+    out = gpu_attention(q, k, v, kv_start, kv_len, anc, status)
+    torch.cuda.synchronize()
+    qb, kb, vb = W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v)
+    Hkv = k.shape[1]
+    got = out.float().cpu().numpy()
+    if sel is None:
+        ref = orc.tree_attention(qb, kb, vb, kv_start, kv_len, parent, st_h, Hkv)
+        return got, ref, status
+    ref = orc.tree_attention_rows(qb, kb, vb, kv_start, kv_len, parent, st_h, Hkv, sel)
+    got = np.stack([got[b, u, h] for b, u, h in sel])
+    return got, ref, status
+
+
+def _inputs(B, M, Hq, Hkv, D, P, seed, left_padded=False, tree="uniform", max_depth=1000, slack=5):
+    rng = np.random.default_rng(seed)
+    g = W.torch_generator(seed, dev())
+    if np.isscalar(P):
+        P = np.full(B, P, np.int32)
+    P = np.asarray(P, np.int32)
+    pmax = int(P.max())
+    kv_start = (pmax - P).astype(np.int32) if left_padded else np.zeros(B, np.int32)
+    S_cap = pmax + M + 1 + slack
+    if tree == "chain":
+        parent = np.stack([W.tree_chain(M)] * B)
+    else:
+        parent = np.stack([W.tree_uniform_depth(M, max_depth, rng) for _ in range(B)])
+    q = W.randn_bf16((B, M + 1, Hq, D), g, dev())
+    k = W.randn_bf16((B, Hkv, S_cap, D), g, dev())
+    v = W.randn_bf16((B, Hkv, S_cap, D), g, dev())
+    return q, k, v, parent.astype(np.int32), kv_start, P.copy()
+
+
+@pytest.mark.parametrize(
+    "B,M,Hq,Hkv,D,P",
+    [
+        (1, 16, 4, 4, 64, 128),  # tiny
+        (1, 0, 4, 4, 64, 77),  # single node = decode
+        (2, 5, 8, 2, 128, 0),  # empty prefix: tree only
+        (3, 9, 6, 3, 64, [1, 100, 333]),  # ragged, odd G
+        (1, 31, 16, 16, 128, 1000),
+        (2, 33, 8, 1, 128, 500),  # MQA, two mask words
+        (1, 255, 2, 1, 128, 200),  # largest tree
+        (4, 20, 12, 4, 128, [64, 65, 127, 129]),  # tile edges
+    ],
+)
+def test_parity_full(orc, B, M, Hq, Hkv, D, P):
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, P, seed=B * 1000 + M)
+    got, ref, _ = _run(orc, q, k, v, par, ks, kl)
+    assert not np.isnan(got).any()
+    assert_attn_close(got, ref, "attention")
+
+
+def test_left_padded_ragged(orc):
+    q, k, v, par, ks, kl = _inputs(5, 7, 16, 4, 128, [10, 700, 64, 1, 1500], seed=3, left_padded=True)
+    got, ref, _ = _run(orc, q, k, v, par, ks, kl)
+    assert_attn_close(got, ref, "left-padded attention")
+
+
+def test_garbage_outside_key_range_is_ignored(orc):
+    """Pad columns and columns past the tree rows hold Inf/NaN: nothing may leak."""
+    B, M, Hq, Hkv, D = 3, 6, 4, 2, 128
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, [5, 90, 40], seed=5, left_padded=True, slack=70)
+    ref_k, ref_v = k.clone(), v.clone()
+    for b in range(B):
+        lo, hi = int(ks[b]), int(ks[b] + kl[b] + M + 1)
+        k[b, :, :lo] = float("nan")
+        v[b, :, :lo] = float("inf")
+        k[b, :, hi:] = float("inf")
+        v[b, :, hi:] = float("nan")
+    got, _, _ = _run(orc, q, k, v, par, ks, kl)
+    _, ref, _ = _run(orc, q, ref_k, ref_v, par, ks, kl)
+    assert np.isfinite(got).all()
+    assert_attn_close(got, ref, "attention with garbage outside the key range")
+
+
+@pytest.mark.parametrize("P", [0, 3, 200])
+def test_no_leak_between_branches(orc, P):
+    B, M, Hq, Hkv, D = 1, 40, 4, 2, 128
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, P, seed=11)
+    _, anc, _, status = gpu_mask(par, 1000)
+    anc_h = anc.cpu().numpy().view(np.uint32)
+    base = gpu_attention(q, k, v, ks, kl, anc, status).float().cpu().numpy()
+    for u in (0, 7, 23, 40):
+        vv = v.clone()
+        for r in range(M + 1):
+            if not (int(anc_h[0, u, r // 32]) >> (r % 32)) & 1:
+                vv[0, :, P + r] = 1e4
+        o = gpu_attention(q, k, vv, ks, kl, anc, status).float().cpu().numpy()
+        np.testing.assert_array_equal(o[0, u], base[0, u])
+
+
+def test_invalid_sequences_zero_rows(orc):
+    B, M, Hq, Hkv, D = 4, 10, 8, 4, 128
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, 300, seed=2)
+    par[1, 3] = 7  # forward pointer: flagged by the mask kernel
+    kl_bad = kl.copy()
+    kl_bad[2] = 10_000  # tree rows would run past the cache
+    got, ref, status = _run(orc, q, k, v, par, ks, kl_bad)
+    assert not got[1].any() and not got[2].any()
+    assert_attn_close(got, ref, "attention with invalid sequences")
+
+
+@pytest.mark.parametrize("name", ["tiny", "mha7b", "eqspec"])
+def test_config_full(orc, name):
+    cfg = W.CONFIGS[name]
+    st = W.make_step(cfg, seed=0, device=dev(), with_logits=False)
+    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth)
+    assert_attn_close(got, ref, name)
+
+
+@pytest.mark.parametrize("name", ["b32gqa", "stress"])
+def test_config_sampled(orc, name):
+    cfg = W.CONFIGS[name]
+    st = W.make_step(cfg, seed=0, device=dev(), with_logits=False)
+    rng = np.random.default_rng(1)
+    n = cfg.M + 1
+    sel = [(0, u, h) for u in range(n) for h in range(0, cfg.Hq, max(1, cfg.Hq // 8))]
+    sel += [(int(rng.integers(cfg.B)), int(rng.integers(n)), int(rng.integers(cfg.Hq))) for _ in range(96)]
+    sel = np.array(sel, np.int32)
+    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth, sel=sel)
+    assert_attn_close(got, ref, name)

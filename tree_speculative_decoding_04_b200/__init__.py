@@ -1,0 +1,24 @@
+"""Teacher-side verification step of tree speculative decoding on NVIDIA B200.
+
+Four calls, each a hand-written sm_100a CUDA kernel behind a C ABI
+(``include/treeverify.h``): ``tree_build_mask``, ``tree_attention``,
+``tree_accept`` and ``kv_commit_realign``.  This package only marshals torch
+tensors into those calls (``_lib``) and offers a host-side driver of one whole
+verification step (``verifier``).
+"""
+from ._lib import (  # noqa: F401
+    EXPORTS,
+    LIB_PATH,
+    MAX_TREE_ROWS,
+    SEQ_BAD_GEOMETRY,
+    SEQ_BAD_PARENT,
+    SEQ_TIMEOUT,
+    SEQ_TOO_DEEP,
+    TVError,
+    kv_commit_realign,
+    layer_pointers,
+    load,
+    tree_accept,
+    tree_attention,
+    tree_build_mask,
+)

@@ -233,14 +233,18 @@ def tagged_rows(layer: int, kvsel: int, B: int, Hkv: int, S_cap: int, D: int, de
     """A [B][Hkv][S_cap][D] bf16 tensor whose every 16-bit word is a hash of
     (salt, layer, K|V, b, h, column, d), with exponent-all-ones patterns (Inf/NaN)
     remapped to finite values, so each moved row proves where it came from."""
-    idx = torch.arange(B * Hkv * S_cap * D, device=device, dtype=torch.int64)
+    out = torch.empty((B, Hkv, S_cap, D), dtype=torch.int16, device=device)
     base = ((salt * 131 + layer) * 2 + kvsel) * 1_000_003
-    h = _mix32_torch(idx * 2654435761 % (1 << 32) + base)
-    bits = (h & 0xFFFF).to(torch.int32)
-    bad = (bits & 0x7F80) == 0x7F80
-    bits = torch.where(bad, bits & ~0x0080, bits)
-    bits = torch.where(bits >= 0x8000, bits - 0x10000, bits).to(torch.int16)
-    return bits.view(torch.bfloat16).reshape(B, Hkv, S_cap, D)
+    per_b = Hkv * S_cap * D
+    for b in range(B):  # one sequence at a time keeps the int64 temporaries small
+        idx = torch.arange(b * per_b, (b + 1) * per_b, device=device, dtype=torch.int64)
+        h = _mix32_torch(idx * 2654435761 % (1 << 32) + base)
+        bits = (h & 0xFFFF).to(torch.int32)
+        bad = (bits & 0x7F80) == 0x7F80
+        bits = torch.where(bad, bits & ~0x0080, bits)
+        bits = torch.where(bits >= 0x8000, bits - 0x10000, bits).to(torch.int16)
+        out[b] = bits.reshape(Hkv, S_cap, D)
+    return out.view(torch.bfloat16)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
