@@ -63,6 +63,7 @@ __device__ __forceinline__ Best warp_best(Best b) {
 __global__ void __launch_bounds__(kArgmaxThreads) accept_argmax_kernel(const float* __restrict__ logits, int V,
                                                                        int chunk, int nsplit,
                                                                        int32_t* __restrict__ argmax_out) {
+  pdl_wait_primary();
   pdl_launch_dependents();
   __shared__ Best warp_res[kArgmaxThreads / 32];
   __shared__ Best cta_res;
@@ -144,7 +145,10 @@ __global__ void __launch_bounds__(kMaxRows) accept_walk_kernel(
   const int64_t rbase = (int64_t)b * n;
   int32_t* pth = path + (int64_t)b * (max_depth + 1);
 
-  // inputs not produced by the argmax kernel: read before waiting on it
+  // Inputs not produced by the argmax kernel may be read before waiting on it:
+  // the argmax kernel triggers this launch only after its own wait returned,
+  // so everything launched before it has completed.
+  pdl_launch_dependents();
   const bool in = u < n;
   const int st0 = status[b];
   const int p = in ? parent[rbase + u] : 0;
@@ -227,7 +231,7 @@ extern "C" tv_status tree_accept(const float* logits, const int32_t* draft, cons
   nsplit = (V + chunk - 1) / chunk;
   if (rows * nsplit > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
   tv_status r = launch(accept_argmax_kernel, dim3((unsigned)(rows * nsplit)), dim3(kArgmaxThreads), 0, s, nsplit,
-                       false, logits, V, chunk, nsplit, argmax);
+                       true, logits, V, chunk, nsplit, argmax);
   if (r != TV_OK) return r;
   const int threads = 32 * ((M + 1 + 31) / 32);
   return launch(accept_walk_kernel, dim3(B), dim3(threads), 0, s, 1, true, (const int32_t*)argmax, draft, parent,

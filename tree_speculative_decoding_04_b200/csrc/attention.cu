@@ -104,14 +104,6 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_kernel(const 
   const int b = bh / p.Hkv;
   const int hk = bh - b * p.Hkv;
 
-  const int32_t ks = p.kv_start[b];
-  const int32_t kl = p.kv_len[b];
-  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
-  const int N = kl + p.M + 1;  // keys of this sequence
-  const int t0 = split * p.tiles_per_split;
-  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + KT - 1) / KT - t0)) : 0;
-  const int k_lo = t0 * KT;
-
   if (threadIdx.x == 0) {
     timed_out = 0;
     for (int s = 0; s < stages; ++s) {
@@ -120,13 +112,26 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_kernel(const 
     }
     fence_mbar_init();
   }
+  if (warp == ncw && lane == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  // everything above overlaps the previous kernel; inputs are read below
+  pdl_wait_primary();
+  pdl_launch_dependents();
   __syncthreads();
+
+  const int32_t ks = p.kv_start[b];
+  const int32_t kl = p.kv_len[b];
+  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int N = kl + p.M + 1;  // keys of this sequence
+  const int t0 = split * p.tiles_per_split;
+  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + KT - 1) / KT - t0)) : 0;
+  const int k_lo = t0 * KT;
 
   if (warp == ncw) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && ntiles > 0) {
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
       int issued = 0;
       bool to = false;
       for (int i = 0; i < ntiles; ++i) {
@@ -463,7 +468,7 @@ tv_status run(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cuda
   p.stages = lp.stages;
   if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
   dim3 grid(lp.nsplit, lp.tiles_q, p.B * p.Hkv);
-  return launch(tree_attn_kernel<D>, grid, dim3((lp.ncw + 1) * 32), lp.smem, s, lp.nsplit, false, tmk, tmv, p);
+  return launch(tree_attn_kernel<D>, grid, dim3((lp.ncw + 1) * 32), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
 }  // namespace

@@ -88,6 +88,7 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
     const int32_t* __restrict__ status, int max_depth, const int32_t* __restrict__ kv_start,
     const int32_t* __restrict__ kv_len, int realign, int64_t runs, uint8_t* __restrict__ attn_mask,
     int32_t* __restrict__ pos_ids) {
+  pdl_wait_primary();
   pdl_launch_dependents();
   extern __shared__ uint4 tail[];  // [max_depth + 1][D / 8]
   __shared__ int red[kMoveThreads / 32];
@@ -189,6 +190,7 @@ __global__ void __launch_bounds__(kPlanThreads) kv_finalize_kernel(
     int32_t* __restrict__ kv_len, int32_t* __restrict__ max_len) {
   __shared__ int red[kPlanThreads / 32];
   pdl_wait_primary();
+  pdl_launch_dependents();
   const int lmax = batch_new_max(B, M, S_cap, max_depth, realign, path, accept_len, status, kv_start, kv_len, red);
   // every thread finished reading the old values inside batch_new_max (it ends with a barrier)
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
@@ -227,11 +229,11 @@ extern "C" tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* cons
     const size_t smem = (size_t)(max_depth + 1) * D * 2;
     cudaError_t e = cudaFuncSetAttribute(kv_move_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return record_cuda_error(e);
-    tv_status r = launch(kv_move_kernel, dim3((unsigned)(runs + extra)), dim3(kMoveThreads), smem, s, 1, false,
+    tv_status r = launch(kv_move_kernel, dim3((unsigned)(runs + extra)), dim3(kMoveThreads), smem, s, 1, true,
                          k_layers, v_layers, B, Hkv, D, S_cap, M, path, accept_len, (const int32_t*)status, max_depth,
                          (const int32_t*)kv_start, (const int32_t*)kv_len, realign, runs, attn_mask, pos_ids);
     if (r != TV_OK) return r;
   }
-  return launch(kv_finalize_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1, runs + extra > 0, B, M, S_cap, max_depth,
+  return launch(kv_finalize_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1, true, B, M, S_cap, max_depth,
                 realign, path, accept_len, status, kv_start, kv_len, max_len);
 }

@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(128) tb_mask_warp_kernel(const int32_t* __rest
                                                            int max_depth, uint32_t* __restrict__ anc,
                                                            int32_t* __restrict__ depth,
                                                            int32_t* __restrict__ status) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (b >= B) return;  // warp-uniform
@@ -67,6 +69,8 @@ __global__ void __launch_bounds__(kMaxRows) tb_mask_block_kernel(const int32_t* 
   __shared__ uint32_t msk[2][kMaxRows][kMaxRows / 32];
   __shared__ int nxt[2][kMaxRows];
   __shared__ int dep[2][kMaxRows];
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int b = blockIdx.x;
   const int u = threadIdx.x;
   const int n = M + 1;
@@ -126,10 +130,10 @@ extern "C" tv_status tree_build_mask(const int32_t* parent, int B, int M, int ma
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (M + 1 <= 32) {
     const int warps = 4;
-    return launch(tb_mask_warp_kernel, dim3((B + warps - 1) / warps), dim3(32 * warps), 0, s, 1, false, parent, B,
+    return launch(tb_mask_warp_kernel, dim3((B + warps - 1) / warps), dim3(32 * warps), 0, s, 1, true, parent, B,
                   M, max_depth, anc_mask, depth, status);
   }
   const int threads = 32 * ((M + 1 + 31) / 32);
-  return launch(tb_mask_block_kernel, dim3(B), dim3(threads), 0, s, 1, false, parent, M, max_depth, anc_mask, depth,
+  return launch(tb_mask_block_kernel, dim3(B), dim3(threads), 0, s, 1, true, parent, M, max_depth, anc_mask, depth,
                 status);
 }
