@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU work budget of the oracle baseline sample")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling runs only)")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -396,8 +398,9 @@ def run_ours(args, cfg, world, rank, local):
     L = cfg.L
     reps = max(5, args.steps // 2)
     g_attn = capture(lambda: [ver.attention(layer, stream) for layer in range(L)], stream)
-    for _ in range(3):
-        g_attn.replay()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_attn.replay()
     attn_ms = event_time(g_attn.replay, reps, stream) / L
     g_mask = capture(lambda: ver.build_mask(stream), stream)
     mask_ms = event_time(g_mask.replay, reps, stream)
@@ -413,6 +416,19 @@ def run_ours(args, cfg, world, rank, local):
     g_reset = capture(reset, stream)
     reset_ms = event_time(g_reset.replay, reps, stream)
     com_ms = max(com_ms - reset_ms, 1e-6)
+
+    # one attention launch alone (eager, not overlapped with a neighbour), median of 20
+    singles = []
+    for r in range(20):
+        with torch.cuda.stream(stream):
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            ver.attention(r % L, stream)
+            a1.record(stream)
+        a1.synchronize()
+        singles.append(a0.elapsed_time(a1))
+    attn_single_ms = statistics.median(singles)
 
     hbm, tflops, peak_kind = peaks()
     a_bytes = attention_bytes(cfg, kl_h)
@@ -431,6 +447,23 @@ def run_ours(args, cfg, world, rank, local):
                  "frac_hbm": c_bytes / (com_ms * 1e-3) / 1e9 / hbm}
 
     # ---- end to end: pinned host inputs -> device, step, results -> host, every step
+    e2e = run_e2e(args, cfg, ver, host, reset, stream, world, device) if not args.no_e2e else None
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rng = np.random.default_rng(2)
+        probe, _ = cpu_oracle_step(cfg, ver, host, 1, min(1.0, 64.0 / (cfg.B * (cfg.M + 1) * cfg.Hq)), rng)
+        layers = int(max(1, min(cfg.L, args.cpu_seconds / max(probe / cfg.L, 1e-6))))
+        t_step, desc = cpu_oracle_step(cfg, ver, host, layers)
+        cpu = {"value": cfg.B * cfg.M / t_step, "unit": "nodes/s", "cores": 1, "kind": "oracle", "sample": desc,
+               "host_threads_available": os.cpu_count()}
+    return finish(args, cfg, world, rank, value, ms_step, roofline, kv_commit, mask_ms, attn_ms, attn_single_ms,
+                  acc_ms, com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device)
+
+
+def run_e2e(args, cfg, ver, host, reset, stream, world, device):
+    L = cfg.L
     h = ver.pinned_inputs()
     h["parent"].copy_(torch.as_tensor(host["parent"]))
     h["draft"].copy_(torch.as_tensor(host["draft"]))
@@ -463,19 +496,13 @@ def run_ours(args, cfg, world, rank, local):
     t1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device) / e2e_steps
-    e2e = {"value": world * cfg.B * cfg.M / (e2e_ms * 1e-3), "unit": "nodes/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": ver.h2d_bytes(), "d2h_bytes_per_step": ver.d2h_bytes()}
+    return {"value": world * cfg.B * cfg.M / (e2e_ms * 1e-3), "unit": "nodes/s", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": ver.h2d_bytes(), "d2h_bytes_per_step": ver.d2h_bytes()}
 
-    # ---- CPU oracle baseline (rank 0, one GPU only)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rng = np.random.default_rng(2)
-        probe, _ = cpu_oracle_step(cfg, ver, host, 1, min(1.0, 64.0 / (cfg.B * (cfg.M + 1) * cfg.Hq)), rng)
-        layers = int(max(1, min(cfg.L, args.cpu_seconds / max(probe / cfg.L, 1e-6))))
-        t_step, desc = cpu_oracle_step(cfg, ver, host, layers)
-        cpu = {"value": cfg.B * cfg.M / t_step, "unit": "nodes/s", "cores": 1, "kind": "oracle", "sample": desc,
-               "host_threads_available": os.cpu_count()}
 
+def finish(args, cfg, world, rank, value, ms_step, roofline, kv_commit, mask_ms, attn_ms, attn_single_ms, acc_ms,
+           com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device):
+    L = cfg.L
     if rank != 0:
         return
     accept_stats = {"mean_accept_len": float(np.mean(al)), "accept_len": al.tolist()}
@@ -491,7 +518,8 @@ def run_ours(args, cfg, world, rank, local):
         "roofline": roofline,
         "kv_commit": kv_commit,
         "breakdown_us": {"tree_build_mask": mask_ms * 1e3, "tree_attention_per_layer": attn_ms * 1e3,
-                         "tree_attention_all_layers": attn_ms * 1e3 * L, "tree_accept": acc_ms * 1e3,
+                         "tree_attention_all_layers": attn_ms * 1e3 * L,
+                         "tree_attention_single_launch": attn_single_ms * 1e3, "tree_accept": acc_ms * 1e3,
                          "kv_commit_realign": com_ms * 1e3, "geometry_reset_copies": reset_ms * 1e3},
         "accept": accept_stats,
         "cpu_baseline": cpu,
@@ -506,6 +534,10 @@ def run_ours(args, cfg, world, rank, local):
 def main():
     args = parse()
     cfg = W.CONFIGS[args.config]
+    if args.layers > 0:
+        import dataclasses
+
+        cfg = dataclasses.replace(cfg, L=args.layers)
     world, rank, local = dist_setup(args) if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")))
     try:
