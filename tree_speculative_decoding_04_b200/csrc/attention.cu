@@ -22,33 +22,18 @@
 #include <algorithm>
 #include <mutex>
 
-#include "tv_common.cuh"
+#include "attention_common.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace tv {
 namespace {
 
-constexpr int KT = 64;          // keys per pipeline stage
+constexpr int KT = kKeyTile;
 constexpr int kMaxCWarps = 8;   // consumer warps per CTA (16 query rows each)
 constexpr int kMaxSplit = 8;    // portable cluster size
-constexpr int kBoxBytes = KT * 128;  // one 64-row x 128-byte swizzled TMA box
 
-struct AttnParams {
-  const uint16_t* q;
-  const int32_t* kv_start;
-  const int32_t* kv_len;
-  const uint32_t* anc;
-  int32_t* status;
-  uint16_t* out;
-  int64_t S_cap;
-  int B, M, Hq, Hkv, G, W;
-  int rows_total;       // G * (M + 1) query rows per (sequence, kv head)
-  int nsplit;           // key splits (cluster size along x)
-  int tiles_per_split;  // 64-key tiles per split
-  int stages;
-  float scale_log2;     // softmax scale * log2(e)
-};
+
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -77,7 +62,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 template <int D>
-__global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                          const __grid_constant__ CUtensorMap tmv,
                                                                          const __grid_constant__ AttnParams p) {
   constexpr int kTileBytes = KT * D * 2;
@@ -377,38 +362,6 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_kernel(const 
   if (threadIdx.x == 0 && timed_out) atomicOr(&p.status[b], kSeqTimeout);
 }
 
-// ---------------------------------------------------------------- host helpers
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-// [B*Hkv][S_cap][D] bf16 -> boxes of 64 columns (128 B) x 64 rows, 128-byte swizzle.
-bool encode_kv_map(CUtensorMap* map, const void* base, int BH, int64_t S_cap, int D) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S_cap, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S_cap * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)KT, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 struct LaunchPlan {
   int ncw, tiles_q, nsplit, tiles_per_split, stages;
   size_t smem;
@@ -437,7 +390,7 @@ tv_status plan_launch(const AttnParams& p, LaunchPlan& lp) {
   // deepest ring that still keeps the whole grid resident (when it can be)
   const int64_t ctas = units * lp.nsplit;
   const int threads = (lp.ncw + 1) * 32;
-  auto kern = tree_attn_kernel<D>;
+  auto kern = tree_attn_mma_kernel<D>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<D>(6));
   if (e != cudaSuccess) return record_cuda_error(e);
   int occ2 = 0;
@@ -468,7 +421,7 @@ tv_status run(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cuda
   p.stages = lp.stages;
   if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
   dim3 grid(lp.nsplit, lp.tiles_q, p.B * p.Hkv);
-  return launch(tree_attn_kernel<D>, grid, dim3((lp.ncw + 1) * 32), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
+  return launch(tree_attn_mma_kernel<D>, grid, dim3((lp.ncw + 1) * 32), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
 }  // namespace
@@ -507,5 +460,6 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
   if (!encode_kv_map(&tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&tmv, v, B * Hkv, S_cap, D))
     return TV_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return D == 64 ? run<64>(tmk, tmv, p, s) : run<128>(tmk, tmv, p, s);
+  // head dim 128 runs on the tcgen05 tensor-core kernel; 64 on the warp-MMA kernel
+  return D == 64 ? run<64>(tmk, tmv, p, s) : run_attention_tc(tmk, tmv, p, s);
 }

@@ -1,0 +1,65 @@
+// attention_common.cuh -- pieces shared by the two tree-attention kernels:
+// launch parameters and the TMA descriptor of one KV-cache layer.
+#pragma once
+
+#include <mutex>
+
+#include "tv_common.cuh"
+
+namespace tv {
+
+constexpr int kKeyTile = 64;             // keys per pipeline stage
+constexpr int kBoxBytes = kKeyTile * 128;  // one 64-row x 128-byte swizzled TMA box
+
+struct AttnParams {
+  const uint16_t* q;
+  const int32_t* kv_start;
+  const int32_t* kv_len;
+  const uint32_t* anc;
+  int32_t* status;
+  uint16_t* out;
+  int64_t S_cap;
+  int B, M, Hq, Hkv, G, W;
+  int rows_total;       // G * (M + 1) query rows per (sequence, kv head)
+  int nsplit;           // key splits (cluster size along x)
+  int tiles_per_split;  // 64-key tiles per split
+  int stages;
+  float scale_log2;     // softmax scale * log2(e)
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// [B*Hkv][S_cap][D] bf16 -> boxes of 64 columns (128 B) x 64 rows, 128-byte swizzle.
+inline bool encode_kv_map(CUtensorMap* map, const void* base, int BH, int64_t S_cap, int D) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S_cap, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S_cap * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kKeyTile, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+
+// Tensor-core (tcgen05) path for head dim 128; defined in attention_tc.cu.
+tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cudaStream_t s);
+
+}  // namespace tv

@@ -1,0 +1,537 @@
+// attention_tc.cu -- tree_attention on the 5th-generation tensor cores
+// (tcgen05 + TMEM) for head dim 128.
+//
+// "EAGLE-Pangu: Accelerator-Safe Tree Speculative Decoding on Ascend NPUs",
+// methodology C: one batched teacher pass over all speculative tokens with a
+// tree mask (node k attends node j only if j is an ancestor of k).  The mask is
+// applied from the ancestor bitmask on the last M+1 key columns only.
+//
+// One CTA owns 128 query rows (tree node x q head of one GQA group) of one
+// (sequence, kv head) and one split of the key range; the splits of a query
+// tile form a thread-block cluster and merge through distributed shared memory.
+// Warp roles (192 threads):
+//   warp 0      TMA producer: 64-key K and V tiles into a 2-stage smem ring
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_i = Q K_i^T   (M=128, N=64, K=128; A, B from smem)   -> TMEM S[i%2]
+//                 O  += P_i V_i   (M=128, N=128, K=64; A=P from TMEM, B=V from smem) -> TMEM O
+//               S_{i+1} is issued before waiting for P_i, so the tensor core
+//               computes the next scores while the softmax warps work.
+//   warps 2-5   softmax: thread t owns TMEM lane t, i.e. query row t; it reads
+//               its 64 scores with one tcgen05.ld, keeps the running max / sum,
+//               writes P (bf16) over its scores, and rescales its O row only
+//               when the running max grows by more than 2^8 (otherwise the
+//               stale max keeps every P <= 256, exact in fp32 accumulation).
+// TMEM: S0 cols [0,64), S1 [64,128), O [128,256); P_i aliases S[i%2] cols [0,32).
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "attention_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace tv {
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kRows = 128;
+constexpr int kTmemCols = 256;
+constexpr int kStages = 2;
+constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
+constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
+constexpr int kStageBytes = 2 * kTileBytes;
+constexpr float kRescaleThreshold = 8.0f;        // log2 domain
+constexpr int kMaxSplit_tc = 8;                  // portable cluster size
+
+// ------------------------------------------------------------------ tcgen05 wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// D (TMEM) (+)= A (smem) * B (smem)
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D (TMEM) (+)= A (TMEM) * B (smem)
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive 32-bit columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle, 8-row groups 1024 B apart.
+// K-major operands (rows of 128 B along K) use lbo = 16 B (unused); the
+// MN-major V operand uses lbo = distance between its two 64-column boxes.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_bytes) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= 1ull << 46;  // descriptor version for sm_100
+  d |= 2ull << 61;  // 128-byte swizzle
+  return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+struct TcSmem {
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_ready[2];  // PV_j completes a phase of o_ready[j % 2]
+  uint64_t q_ready;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int timed_out;
+  float m_st[kRows];
+  float l_st[kRows];
+};
+
+// O += P_j V_j for key tile j (one thread), then release the K/V stage and
+// publish the new O.  Returns false if P_j never arrived.
+__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t t_s0, uint32_t t_o, int j) {
+  const uint32_t idesc_o = idesc_bf16(128, 128, 1);
+  const int sb = j & 1, s = j % kStages;
+  if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1)) return false;
+  tc_fence_after();
+  const uint32_t v_addr = smem_u32(stage_s + s * kStageBytes + kTileBytes);
+#pragma unroll
+  for (int kk = 0; kk < kKeyTile / 16; ++kk)
+    mma_ts(t_o, t_s0 + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
+           (j > 0 || kk > 0) ? 1u : 0u);
+  tc_commit(&sh->kv_empty[s]);
+  tc_commit(&sh->o_ready[j & 1]);
+  return true;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                                                                    const __grid_constant__ CUtensorMap tmv,
+                                                                    const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem;                              // [2][128][128 B]
+  uint8_t* stage_s = smem + kQBytes;                // [kStages][K box0, K box1, V box0, V box1]
+  TcSmem* sh = reinterpret_cast<TcSmem*>(stage_s + kStages * kStageBytes);
+  float* o_stage = reinterpret_cast<float*>(smem);  // [128][128] fp32 after the MMAs are done
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int qtile = blockIdx.y;
+  const int bh = blockIdx.z;
+  const int b = bh / p.Hkv;
+  const int hk = bh - b * p.Hkv;
+
+  if (threadIdx.x == 0) {
+    sh->timed_out = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sh->kv_full[s], 1);
+      mbar_init(&sh->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh->s_full[s], 1);
+      mbar_init(&sh->p_full[s], 4);
+    }
+    mbar_init(&sh->o_ready[0], 1);
+    mbar_init(&sh->o_ready[1], 1);
+    mbar_init(&sh->q_ready, 4);
+    mbar_init(&sh->drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  if (warp == 1) {
+    tmem_alloc(&sh->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t t_s0 = tmem, t_o = tmem + 128;
+
+  const int32_t ks = p.kv_start[b];
+  const int32_t kl = p.kv_len[b];
+  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int N = kl + p.M + 1;
+  const int t0 = split * p.tiles_per_split;
+  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + kKeyTile - 1) / kKeyTile - t0)) : 0;
+  const int k_lo = t0 * kKeyTile;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool to = false;
+      int issued = 0;
+      for (int i = 0; i < ntiles && !to; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&sh->kv_empty[s], ((i / kStages) - 1) & 1)) {
+          to = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&sh->kv_full[s], kStageBytes);
+        const int col = ks + k_lo + i * kKeyTile;
+        uint8_t* st = stage_s + s * kStageBytes;
+        tma_load_3d(st, &tmk, &sh->kv_full[s], 0, col, bh);
+        tma_load_3d(st + kBoxBytes, &tmk, &sh->kv_full[s], 64, col, bh);
+        tma_load_3d(st + kTileBytes, &tmv, &sh->kv_full[s], 0, col, bh);
+        tma_load_3d(st + kTileBytes + kBoxBytes, &tmv, &sh->kv_full[s], 64, col, bh);
+        ++issued;
+      }
+      if (to) {
+        atomicExch(&sh->timed_out, 1);
+        // copies still in flight must land before this CTA's shared memory is released
+        for (int i = max(0, issued - kStages); i < issued; ++i) mbar_wait(&sh->kv_full[i % kStages], (i / kStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
+      const uint32_t q_addr = smem_u32(q_s);
+      bool to = !mbar_wait(&sh->q_ready, 0);
+      tc_fence_after();
+      for (int i = 0; i < ntiles && !to; ++i) {
+        const int s = i % kStages, sb = i & 1;
+        if (!mbar_wait(&sh->kv_full[s], (i / kStages) & 1)) {
+          to = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(stage_s + s * kStageBytes);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
+          const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
+          mma_ss(t_s0 + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&sh->s_full[sb]);
+        if (i >= 1 && !issue_pv(sh, stage_s, t_s0, t_o, i - 1)) to = true;
+      }
+      if (!to && !issue_pv(sh, stage_s, t_s0, t_o, ntiles - 1)) to = true;
+      if (to) {
+        atomicExch(&sh->timed_out, 1);
+        // let every MMA issued so far retire before TMEM and shared memory are released
+        tc_commit(&sh->drain);
+        mbar_wait(&sh->drain, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps
+    const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int gr = qtile * kRows + r;
+    const bool row_ok = gr < p.rows_total;
+    const int u = min(gr / p.G, p.M);
+    const int hq = hk * p.G + gr % p.G;
+    // Q row -> swizzled smem (two 64-column boxes), zero rows past the tile
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * (p.M + 1) + u) * p.Hq + hq) * 128);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row_ok) v = __ldg(src + c);
+        *reinterpret_cast<uint4*>(q_s + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->q_ready);
+    }
+    uint32_t anc_w[kMaxRows / 32];
+#pragma unroll
+    for (int w = 0; w < kMaxRows / 32; ++w)
+      anc_w[w] = w < p.W ? __ldg(p.anc + ((int64_t)b * (p.M + 1) + u) * p.W + w) : 0u;
+
+    float m = -INFINITY, l = 0.f;
+    bool to = false;
+    for (int i = 0; i < ntiles; ++i) {
+      const int sb = i & 1;
+      if (!mbar_wait(&sh->s_full[sb], (i >> 1) & 1)) {
+        to = true;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(t_s0 + lane_off + sb * 64, sr[0]);
+      tmem_ld32(t_s0 + lane_off + sb * 64 + 32, sr[1]);
+      tmem_wait_ld();
+      const int key0 = k_lo + i * kKeyTile;
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 64; ++j) {
+        float v = __uint_as_float(sr[j >> 5][j & 31]) * p.scale_log2;
+        x[j] = v;
+      }
+      if (key0 + kKeyTile > kl) {  // tile reaches the tree rows or the end of the range
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int key = key0 + j;
+          bool ok = key < kl;
+          if (!ok && key < N) {
+            const int t = key - kl;
+            uint32_t w = 0;
+#pragma unroll
+            for (int q = 0; q < kMaxRows / 32; ++q) w = (q == (t >> 5)) ? anc_w[q] : w;
+            ok = (w >> (t & 31)) & 1u;
+          }
+          if (!ok) x[j] = -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 64; ++j) mx = fmaxf(mx, x[j]);
+      if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
+        if (m != -INFINITY) {
+          // O holds data from earlier tiles: rescale this row once PV_{i-1} has landed
+          const float corr = fast_exp2(m - mx);
+          if (!mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+            to = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+            tmem_st32(t_o + lane_off + c * 32, o);
+          }
+          tmem_wait_st();
+          l *= corr;
+        }
+        m = mx;
+      }
+      const float ms = m == -INFINITY ? 0.f : m;
+      uint32_t pk[32];
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float p0 = fast_exp2(x[2 * j] - ms), p1 = fast_exp2(x[2 * j + 1] - ms);
+        rs += p0 + p1;
+        pk[j] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      // past the end of the key range the V rows may hold anything: zero them
+      const int kend = N - key0;
+      if (kend < kKeyTile) {
+        uint8_t* vt = stage_s + (i % kStages) * kStageBytes + kTileBytes;
+        const int first = max(kend, 0);
+        for (int idx = r; idx < (kKeyTile - first) * 16; idx += kRows) {
+          const int row = first + idx / 16, c = idx % 16;
+          *reinterpret_cast<uint4*>(vt + (c >> 3) * kBoxBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
+              make_uint4(0, 0, 0, 0);
+        }
+        fence_async_smem();
+      }
+      tmem_st32(t_s0 + lane_off + sb * 64, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->p_full[sb]);
+    }
+    if (to) atomicExch(&sh->timed_out, 1);
+
+    // ------------------------------------------------------------------ epilogue
+    const bool have = ntiles > 0 && !to;
+    if (have) {
+      if (!mbar_wait(&sh->o_ready[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1)) {
+        atomicExch(&sh->timed_out, 1);
+      }
+      tc_fence_after();
+    }
+    const int64_t orow = (((int64_t)b * (p.M + 1) + gr / p.G) * p.Hq + hq) * 128;
+    if (p.nsplit == 1) {
+      const float inv = (have && valid && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(t_o + lane_off + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + orow + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+            dst[q4] = w;
+          }
+        }
+      }
+    } else {
+      // partial (max, sum, unnormalised O) of this split -> own smem for the cluster merge
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(t_o + lane_off + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+        float4* dst = reinterpret_cast<float4*>(o_stage + r * 128 + c * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          // rotate the 16-byte slots by row to spread shared-memory banks
+          const int slot = (q4 + r) & 7;
+          dst[slot] = make_float4(__uint_as_float(o[4 * slot]), __uint_as_float(o[4 * slot + 1]),
+                                  __uint_as_float(o[4 * slot + 2]), __uint_as_float(o[4 * slot + 3]));
+        }
+      }
+      sh->m_st[r] = have ? m : -INFINITY;
+      sh->l_st[r] = have ? l : 0.f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (p.nsplit > 1) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int ns = p.nsplit;
+    const int rank = (int)cluster.block_rank();
+    const int r_lo = rank * kRows / ns, r_hi = (rank + 1) * kRows / ns;
+    for (int idx = threadIdx.x; idx < (r_hi - r_lo) * 32; idx += blockDim.x) {
+      const int rr = r_lo + idx / 32;
+      const int d = (idx % 32) * 4;
+      const int g2 = qtile * kRows + rr;
+      if (g2 >= p.rows_total) continue;
+      float mj[kMaxSplit_tc], lj[kMaxSplit_tc];
+      float4 oj[kMaxSplit_tc];
+#pragma unroll
+      for (int j = 0; j < kMaxSplit_tc; ++j) {
+        if (j < ns) {
+          const TcSmem* peer = cluster.map_shared_rank(sh, (unsigned)j);
+          mj[j] = peer->m_st[rr];
+          lj[j] = peer->l_st[rr];
+          oj[j] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(o_stage, (unsigned)j) + rr * 128 + d);
+        } else {
+          mj[j] = -INFINITY;
+          lj[j] = 0.f;
+          oj[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      float mmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMaxSplit_tc; ++j) mmax = fmaxf(mmax, mj[j]);
+      const float msafe = mmax == -INFINITY ? 0.f : mmax;
+      float L = 0.f;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < kMaxSplit_tc; ++j) {
+        const float w = fast_exp2(mj[j] - msafe);
+        L += w * lj[j];
+        a.x += w * oj[j].x;
+        a.y += w * oj[j].y;
+        a.z += w * oj[j].z;
+        a.w += w * oj[j].w;
+      }
+      const float inv = (valid && L > 0.f) ? 1.f / L : 0.f;
+      const int64_t orow = (((int64_t)b * (p.M + 1) + g2 / p.G) * p.Hq + hk * p.G + g2 % p.G) * 128;
+      uint2 pk;
+      pk.x = pack_bf16x2(a.x * inv, a.y * inv);
+      pk.y = pack_bf16x2(a.z * inv, a.w * inv);
+      *reinterpret_cast<uint2*>(p.out + orow + d) = pk;
+    }
+    cluster.sync();  // peers may still be reading this CTA's shared memory
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && sh->timed_out) atomicOr(&p.status[b], kSeqTimeout);
+}
+
+}  // namespace
+
+tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles_q = (p.rows_total + kRows - 1) / kRows;
+  const int64_t units = (int64_t)p.B * p.Hkv * tiles_q;
+  const int key_tiles = (int)std::max<int64_t>(1, (p.S_cap + kKeyTile - 1) / kKeyTile);
+  int ns = (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms + units - 1) / units));
+  ns = std::min(ns, key_tiles);
+  p.tiles_per_split = (key_tiles + ns - 1) / ns;
+  p.nsplit = (key_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  p.stages = kStages;
+  // At most two CTAs per SM: each holds 256 of the 512 TMEM columns, so an
+  // allocation never waits on a CTA that is itself waiting.
+  const size_t smem = 1024 + kQBytes + (size_t)kStages * kStageBytes + sizeof(TcSmem);
+  e = cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tree_attn_tc_kernel, kTcThreads, smem);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (occ > 2 || occ < 1) return TV_ERR_UNSUPPORTED;
+  if ((int64_t)p.B * p.Hkv > 65535 || tiles_q > 65535) return TV_ERR_UNSUPPORTED;
+  dim3 grid(p.nsplit, tiles_q, p.B * p.Hkv);
+  return launch(tree_attn_tc_kernel, grid, dim3(kTcThreads), smem, s, p.nsplit, true, tmk, tmv, p);
+}
+
+}  // namespace tv
