@@ -98,18 +98,26 @@ tv_status tree_build_mask(const int32_t* parent, int B, int M, int max_depth, ui
  *   k, v      bf16 [B][Hkv][S_cap][D]    in (one layer); 16-byte aligned
  *   kv_start, kv_len  int32 [B]          in
  *   anc_mask  uint32 [B][M+1][W]         in (from tree_build_mask)
- *   status    int32 [B]                  in/out: sequences with status != 0 are
- *             skipped (zero output); bad geometry / wait timeouts are OR-ed in
+ *   status    int32 [B]                  in/out: sequences with status != 0 (or a
+ *             bad cache geometry) get zero output rows; a device wait that timed
+ *             out ORs in TV_SEQ_TIMEOUT
  *   out       bf16 [B][M+1][Hq][D]       out: softmax(q k^T * scale) v over the
  *             allowed keys, fp32 accumulation
+ *   workspace device scratch of at least tree_attention_workspace_size(...)
+ *             bytes (16-byte aligned; may be NULL when that size is 0).  It holds
+ *             the partial results of the key splits of one call; its contents
+ *             need no initialisation and are dead after the call.  Calls that
+ *             overlap on the device must not share a workspace.
  *   D in {64, 128}; Hq % Hkv == 0 (q head h reads kv head h / (Hq/Hkv));
  *   scale > 0 (normally 1/sqrt(D)).
  * Contract: the K/V rows inside each sequence's key range hold finite values.
  */
+size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64_t S_cap);
+
 tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                          const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                          int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
-                         uint16_t* out, tv_stream_t stream);
+                         uint16_t* out, void* workspace, size_t workspace_bytes, tv_stream_t stream);
 
 /*
  * tree_accept -- per-node greedy argmax of the teacher logits fused with

@@ -15,10 +15,12 @@ from ._lib import (  # noqa: F401
     SEQ_TIMEOUT,
     SEQ_TOO_DEEP,
     TVError,
+    attention_workspace,
     kv_commit_realign,
     layer_pointers,
     load,
     tree_accept,
     tree_attention,
+    tree_attention_workspace_size,
     tree_build_mask,
 )

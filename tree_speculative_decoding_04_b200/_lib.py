@@ -24,6 +24,7 @@ MAX_TREE_ROWS = 256
 
 EXPORTS = (
     "tree_build_mask",
+    "tree_attention_workspace_size",
     "tree_attention",
     "tree_accept",
     "kv_commit_realign",
@@ -50,7 +51,9 @@ def load(path: str = LIB_PATH):
     lib = ctypes.CDLL(path)
     P, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
     lib.tree_build_mask.argtypes = [P, i32, i32, i32, P, P, P, P]
-    lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
+    lib.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
+    lib.tree_attention_workspace_size.restype = ctypes.c_size_t
+    lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, ctypes.c_size_t, P]
     lib.tree_accept.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, P]
     lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P]
     for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign"):
@@ -108,8 +111,22 @@ def tree_build_mask(parent, max_depth, anc_mask, depth, status, stream=None):
     _check(rc, "tree_build_mask")
 
 
-def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, scale=None, stream=None):
-    """q [B][M+1][Hq][D] bf16; k, v [B][Hkv][S_cap][D] bf16 (one layer) -> out like q."""
+def tree_attention_workspace_size(B, M, Hq, Hkv, D, S_cap) -> int:
+    """Bytes of device scratch tree_attention needs for this shape (0 = none)."""
+    return int(load().tree_attention_workspace_size(B, M, Hq, Hkv, D, int(S_cap)))
+
+
+def attention_workspace(B, M, Hq, Hkv, D, S_cap, device) -> torch.Tensor | None:
+    """A device buffer of the workspace size (None when no workspace is needed)."""
+    nbytes = tree_attention_workspace_size(B, M, Hq, Hkv, D, S_cap)
+    if nbytes == 0:
+        return None
+    return torch.empty((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+
+def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=None, scale=None, stream=None):
+    """q [B][M+1][Hq][D] bf16; k, v [B][Hkv][S_cap][D] bf16 (one layer) -> out like q.
+    workspace: a uint8 device tensor of at least tree_attention_workspace_size bytes."""
     B, n, Hq, D = q.shape
     Hkv, S_cap = k.shape[1], k.shape[2]
     _need(q, torch.bfloat16, (B, n, Hq, D), "q")
@@ -122,8 +139,10 @@ def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, scale=None,
     _need(out, torch.bfloat16, (B, n, Hq, D), "out")
     if scale is None:
         scale = D ** -0.5
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load().tree_attention(_ptr(q), _ptr(k), _ptr(v), S_cap, _ptr(kv_start), _ptr(kv_len), _ptr(anc_mask),
-                               _ptr(status), B, n - 1, Hq, Hkv, D, float(scale), _ptr(out), _stream(stream))
+                               _ptr(status), B, n - 1, Hq, Hkv, D, float(scale), _ptr(out), _ptr(workspace),
+                               ws_bytes, _stream(stream))
     _check(rc, "tree_attention")
 
 

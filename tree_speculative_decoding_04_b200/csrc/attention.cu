@@ -427,10 +427,19 @@ tv_status run(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cuda
 }  // namespace
 }  // namespace tv
 
+extern "C" size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64_t S_cap) {
+  using namespace tv;
+  if (B <= 0 || M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S_cap < 0 || D != 128) return 0;
+  if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return 0;
+  TcPlan plan;
+  if (plan_attention_tc(B, M, Hq, Hkv, S_cap, plan) != TV_OK) return 0;
+  return plan.ws_bytes;
+}
+
 extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                                     const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                                     int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
-                                    uint16_t* out, tv_stream_t stream) {
+                                    uint16_t* out, void* workspace, size_t workspace_bytes, tv_stream_t stream) {
   using namespace tv;
   if (B < 0 || M < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || !(scale > 0.f)) return TV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return TV_ERR_INVALID_ARG;
@@ -456,10 +465,19 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
   p.rows_total = p.G * (M + 1);
   p.nsplit = p.tiles_per_split = p.stages = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.ws = nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   CUtensorMap tmk, tmv;
   if (!encode_kv_map(&tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&tmv, v, B * Hkv, S_cap, D))
     return TV_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // head dim 128 runs on the tcgen05 tensor-core kernel; 64 on the warp-MMA kernel
-  return D == 64 ? run<64>(tmk, tmv, p, s) : run_attention_tc(tmk, tmv, p, s);
+  if (D == 64) return run<64>(tmk, tmv, p, s);  // warp-MMA kernel, merge through DSMEM
+  // head dim 128: tcgen05 tensor-core kernel
+  TcPlan plan;
+  tv_status r = plan_attention_tc(B, M, Hq, Hkv, S_cap, plan);
+  if (r != TV_OK) return r;
+  if (plan.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < plan.ws_bytes || !aligned16(workspace)) return TV_ERR_INVALID_ARG;
+    p.ws = static_cast<float*>(workspace);
+  }
+  return run_attention_tc(tmk, tmv, p, plan, s);
 }

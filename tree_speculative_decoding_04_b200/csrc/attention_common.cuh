@@ -25,6 +25,7 @@ struct AttnParams {
   int tiles_per_split;  // 64-key tiles per split
   int stages;
   float scale_log2;     // softmax scale * log2(e)
+  float* ws;            // split partials: [units][nsplit][128 rows][128] O, then [units][nsplit][128][2] (m, l)
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -60,6 +61,12 @@ inline bool encode_kv_map(CUtensorMap* map, const void* base, int BH, int64_t S_
 
 
 // Tensor-core (tcgen05) path for head dim 128; defined in attention_tc.cu.
-tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cudaStream_t s);
+struct TcPlan {
+  int tiles_q, nsplit, tiles_per_split, stages;
+  size_t smem, ws_bytes;
+};
+tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& plan);
+tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, const TcPlan& plan,
+                           cudaStream_t s);
 
 }  // namespace tv

@@ -36,7 +36,7 @@ namespace {
 constexpr int kTcThreads = 192;
 constexpr int kRows = 128;
 constexpr int kTmemCols = 256;
-constexpr int kStages = 2;
+constexpr int kMaxStages = 6;
 constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
 constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
 constexpr int kStageBytes = 2 * kTileBytes;
@@ -123,8 +123,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) 
 }
 
 struct TcSmem {
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t kv_full[kMaxStages];
+  uint64_t kv_empty[kMaxStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_ready[2];  // PV_j completes a phase of o_ready[j % 2]
@@ -132,15 +132,28 @@ struct TcSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int timed_out;
-  float m_st[kRows];
-  float l_st[kRows];
 };
+
+// bits [start, start + 64) of an ancestor row (bit t = tree row t); rows outside
+// [0, 32 * 8) read as 0, so a window that starts inside the prefix is fine.
+__device__ __forceinline__ uint64_t anc_window(const uint32_t (&aw)[kMaxRows / 32], int start) {
+  uint64_t r = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxRows / 32; ++q) {
+    const int off = q * 32 - start;  // where bit 0 of word q lands in the window
+    const uint64_t w = aw[q];
+    if (off >= 0 && off < 64) r |= w << off;
+    else if (off < 0 && off > -32) r |= w >> (-off);
+  }
+  return r;
+}
 
 // O += P_j V_j for key tile j (one thread), then release the K/V stage and
 // publish the new O.  Returns false if P_j never arrived.
-__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t t_s0, uint32_t t_o, int j) {
+__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t t_s0, uint32_t t_o, int j,
+                                         int stages) {
   const uint32_t idesc_o = idesc_bf16(128, 128, 1);
-  const int sb = j & 1, s = j % kStages;
+  const int sb = j & 1, s = j % stages;
   if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1)) return false;
   tc_fence_after();
   const uint32_t v_addr = smem_u32(stage_s + s * kStageBytes + kTileBytes);
@@ -153,15 +166,15 @@ __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t 
   return true;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                     const __grid_constant__ CUtensorMap tmv,
                                                                     const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_s = smem;                              // [2][128][128 B]
-  uint8_t* stage_s = smem + kQBytes;                // [kStages][K box0, K box1, V box0, V box1]
-  TcSmem* sh = reinterpret_cast<TcSmem*>(stage_s + kStages * kStageBytes);
-  float* o_stage = reinterpret_cast<float*>(smem);  // [128][128] fp32 after the MMAs are done
+  const int stages = p.stages;
+  uint8_t* stage_s = smem + kQBytes;                // [stages][K box0, K box1, V box0, V box1]
+  TcSmem* sh = reinterpret_cast<TcSmem*>(stage_s + stages * kStageBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -173,7 +186,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
 
   if (threadIdx.x == 0) {
     sh->timed_out = 0;
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(&sh->kv_full[s], 1);
       mbar_init(&sh->kv_empty[s], 1);
     }
@@ -183,7 +196,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
     }
     mbar_init(&sh->o_ready[0], 1);
     mbar_init(&sh->o_ready[1], 1);
-    mbar_init(&sh->q_ready, 4);
     mbar_init(&sh->drain, 1);
     fence_mbar_init();
   }
@@ -193,6 +205,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
   }
   pdl_wait_primary();
   pdl_launch_dependents();
+  const int32_t ks = p.kv_start[b];
+  const int32_t kl = p.kv_len[b];
+  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int N = kl + p.M + 1;
+  const int t0 = split * p.tiles_per_split;
+  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + kKeyTile - 1) / kKeyTile - t0)) : 0;
+  const int k_lo = t0 * kKeyTile;
+
+  // The first ring's worth of K/V tiles and the Q tile are requested before the
+  // TMEM allocation barrier, so their memory latency overlaps the set-up.
+  auto issue_kv = [&](int i) {
+    const int s = i % stages;
+    mbar_arrive_expect_tx(&sh->kv_full[s], kStageBytes);
+    const int col = ks + k_lo + i * kKeyTile;
+    uint8_t* st = stage_s + s * kStageBytes;
+    tma_load_3d(st, &tmk, &sh->kv_full[s], 0, col, bh);
+    tma_load_3d(st + kBoxBytes, &tmk, &sh->kv_full[s], 64, col, bh);
+    tma_load_3d(st + kTileBytes, &tmv, &sh->kv_full[s], 0, col, bh);
+    tma_load_3d(st + kTileBytes + kBoxBytes, &tmv, &sh->kv_full[s], 64, col, bh);
+  };
+  const int prologue_tiles = min(ntiles, stages);
+  if (warp == 0 && lane == 0)  // the thread that initialised the barriers
+    for (int i = 0; i < prologue_tiles; ++i) issue_kv(i);
+  const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
+  const int gr = qtile * kRows + r;
+  const bool row_ok = gr < p.rows_total;
+  const int hq = hk * p.G + gr % p.G;
+  const int u = min(gr / p.G, p.M);
+  uint32_t anc_w[kMaxRows / 32];
+  if (warp >= 2) {
+    // Q row -> swizzled smem (two 64-column boxes); rows past the tile are zero
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * (p.M + 1) + u) * p.Hq + hq) * 128);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row_ok) v = __ldg(src + c);
+      *reinterpret_cast<uint4*>(q_s + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+    }
+    fence_async_smem();  // generic-proxy stores -> visible to the tensor core after the barrier
+#pragma unroll
+    for (int w = 0; w < kMaxRows / 32; ++w)
+      anc_w[w] = w < p.W ? __ldg(p.anc + ((int64_t)b * (p.M + 1) + u) * p.W + w) : 0u;
+  }
   if (warp == 1) {
     tmem_alloc(&sh->tmem_base, kTmemCols);
     tmem_relinquish();
@@ -203,38 +258,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
   const uint32_t tmem = sh->tmem_base;
   const uint32_t t_s0 = tmem, t_o = tmem + 128;
 
-  const int32_t ks = p.kv_start[b];
-  const int32_t kl = p.kv_len[b];
-  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
-  const int N = kl + p.M + 1;
-  const int t0 = split * p.tiles_per_split;
-  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + kKeyTile - 1) / kKeyTile - t0)) : 0;
-  const int k_lo = t0 * kKeyTile;
-
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool to = false;
-      int issued = 0;
-      for (int i = 0; i < ntiles && !to; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&sh->kv_empty[s], ((i / kStages) - 1) & 1)) {
+      int issued = prologue_tiles;
+      for (int i = prologue_tiles; i < ntiles && !to; ++i) {
+        const int s = i % stages;
+        if (!mbar_wait(&sh->kv_empty[s], ((i / stages) - 1) & 1)) {
           to = true;
           break;
         }
-        mbar_arrive_expect_tx(&sh->kv_full[s], kStageBytes);
-        const int col = ks + k_lo + i * kKeyTile;
-        uint8_t* st = stage_s + s * kStageBytes;
-        tma_load_3d(st, &tmk, &sh->kv_full[s], 0, col, bh);
-        tma_load_3d(st + kBoxBytes, &tmk, &sh->kv_full[s], 64, col, bh);
-        tma_load_3d(st + kTileBytes, &tmv, &sh->kv_full[s], 0, col, bh);
-        tma_load_3d(st + kTileBytes + kBoxBytes, &tmv, &sh->kv_full[s], 64, col, bh);
+        issue_kv(i);
         ++issued;
       }
       if (to) {
         atomicExch(&sh->timed_out, 1);
         // copies still in flight must land before this CTA's shared memory is released
-        for (int i = max(0, issued - kStages); i < issued; ++i) mbar_wait(&sh->kv_full[i % kStages], (i / kStages) & 1);
+        for (int i = max(0, issued - stages); i < issued; ++i) mbar_wait(&sh->kv_full[i % stages], (i / stages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -242,11 +283,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
     if (lane == 0 && ntiles > 0) {
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
       const uint32_t q_addr = smem_u32(q_s);
-      bool to = !mbar_wait(&sh->q_ready, 0);
-      tc_fence_after();
+      bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
-        const int s = i % kStages, sb = i & 1;
-        if (!mbar_wait(&sh->kv_full[s], (i / kStages) & 1)) {
+        const int s = i % stages, sb = i & 1;
+        if (!mbar_wait(&sh->kv_full[s], (i / stages) & 1)) {
           to = true;
           break;
         }
@@ -259,9 +299,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
           mma_ss(t_s0 + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
         }
         tc_commit(&sh->s_full[sb]);
-        if (i >= 1 && !issue_pv(sh, stage_s, t_s0, t_o, i - 1)) to = true;
+        if (i >= 1 && !issue_pv(sh, stage_s, t_s0, t_o, i - 1, stages)) to = true;
       }
-      if (!to && !issue_pv(sh, stage_s, t_s0, t_o, ntiles - 1)) to = true;
+      if (!to && !issue_pv(sh, stage_s, t_s0, t_o, ntiles - 1, stages)) to = true;
       if (to) {
         atomicExch(&sh->timed_out, 1);
         // let every MMA issued so far retire before TMEM and shared memory are released
@@ -269,33 +309,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
         mbar_wait(&sh->drain, 0);
       }
     }
-  } else {
-    // ------------------------------------------------------------------ softmax warps
-    const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
-    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const int gr = qtile * kRows + r;
-    const bool row_ok = gr < p.rows_total;
-    const int u = min(gr / p.G, p.M);
-    const int hq = hk * p.G + gr % p.G;
-    // Q row -> swizzled smem (two 64-column boxes), zero rows past the tile
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * (p.M + 1) + u) * p.Hq + hq) * 128);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row_ok) v = __ldg(src + c);
-        *reinterpret_cast<uint4*>(q_s + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
-      }
-      fence_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->q_ready);
-    }
-    uint32_t anc_w[kMaxRows / 32];
-#pragma unroll
-    for (int w = 0; w < kMaxRows / 32; ++w)
-      anc_w[w] = w < p.W ? __ldg(p.anc + ((int64_t)b * (p.M + 1) + u) * p.W + w) : 0u;
+  }
 
-    float m = -INFINITY, l = 0.f;
+  // ------------------------------------------------------------------ softmax warps
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  float m = -INFINITY, l = 0.f;
+  bool have = false;
+  const bool warp_live = __any_sync(0xffffffffu, row_ok);  // some row of this warp is real
+  if (warp >= 2) {
     bool to = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1;
@@ -304,72 +325,71 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
         break;
       }
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(t_s0 + lane_off + sb * 64, sr[0]);
-      tmem_ld32(t_s0 + lane_off + sb * 64 + 32, sr[1]);
-      tmem_wait_ld();
       const int key0 = k_lo + i * kKeyTile;
-      float x[64];
-      float mx = -INFINITY;
+      // a warp made only of padding rows (zero queries, so zero scores and a zero
+      // P already in TMEM) has nothing to compute
+      if (warp_live) {
+        uint32_t sr[2][32];
+        tmem_ld32(t_s0 + lane_off + sb * 64, sr[0]);
+        tmem_ld32(t_s0 + lane_off + sb * 64 + 32, sr[1]);
+        tmem_wait_ld();
+        float x[64];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        float v = __uint_as_float(sr[j >> 5][j & 31]) * p.scale_log2;
-        x[j] = v;
-      }
-      if (key0 + kKeyTile > kl) {  // tile reaches the tree rows or the end of the range
+        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sr[j >> 5][j & 31]) * p.scale_log2;
+        if (key0 + kKeyTile > kl) {  // tile reaches the tree rows or the end of the range
+          const int np = kl - key0;  // prefix keys in this tile
+          const uint64_t pre = np >= 64 ? ~0ull : (np <= 0 ? 0ull : ((1ull << np) - 1ull));
+          const uint64_t allowed = pre | anc_window(anc_w, key0 - kl);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int key = key0 + j;
-          bool ok = key < kl;
-          if (!ok && key < N) {
-            const int t = key - kl;
-            uint32_t w = 0;
-#pragma unroll
-            for (int q = 0; q < kMaxRows / 32; ++q) w = (q == (t >> 5)) ? anc_w[q] : w;
-            ok = (w >> (t & 31)) & 1u;
-          }
-          if (!ok) x[j] = -INFINITY;
+          for (int j = 0; j < 64; ++j)
+            if (!((allowed >> j) & 1ull)) x[j] = -INFINITY;
         }
-      }
+        float mx8[8];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) mx = fmaxf(mx, x[j]);
-      if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
-        if (m != -INFINITY) {
-          // O holds data from earlier tiles: rescale this row once PV_{i-1} has landed
-          const float corr = fast_exp2(m - mx);
-          if (!mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-            to = true;
-            break;
+        for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(fmaxf(fmaxf(x[q], x[q + 8]), fmaxf(x[q + 16], x[q + 24])),
+                                                  fmaxf(fmaxf(x[q + 32], x[q + 40]), fmaxf(x[q + 48], x[q + 56])));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
+          if (m != -INFINITY) {
+            // O holds earlier tiles: rescale this row once PV_{i-1} has landed
+            const float corr = fast_exp2(m - mx);
+            if (!mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
+              to = true;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(t_o + lane_off + c * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+              tmem_st32(t_o + lane_off + c * 32, o);
+            }
+            tmem_wait_st();
+            l *= corr;
           }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(t_o + lane_off + c * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
-            tmem_st32(t_o + lane_off + c * 32, o);
-          }
-          tmem_wait_st();
-          l *= corr;
+          m = mx;
         }
-        m = mx;
-      }
-      const float ms = m == -INFINITY ? 0.f : m;
-      uint32_t pk[32];
-      float rs = 0.f;
+        const float ms = m == -INFINITY ? 0.f : m;
+        uint32_t pk[32];
+        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float p0 = fast_exp2(x[2 * j] - ms), p1 = fast_exp2(x[2 * j + 1] - ms);
-        rs += p0 + p1;
-        pk[j] = pack_bf16x2(p0, p1);
+        for (int j = 0; j < 32; ++j) {
+          const float p0 = fast_exp2(x[2 * j] - ms), p1 = fast_exp2(x[2 * j + 1] - ms);
+          rs8[j & 7] += p0 + p1;
+          pk[j] = pack_bf16x2(p0, p1);
+        }
+        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        tmem_st32(t_s0 + lane_off + sb * 64, pk);
+        tmem_wait_st();
       }
-      l += rs;
       // past the end of the key range the V rows may hold anything: zero them
       const int kend = N - key0;
       if (kend < kKeyTile) {
-        uint8_t* vt = stage_s + (i % kStages) * kStageBytes + kTileBytes;
+        uint8_t* vt = stage_s + (i % stages) * kStageBytes + kTileBytes;
         const int first = max(kend, 0);
         for (int idx = r; idx < (kKeyTile - first) * 16; idx += kRows) {
           const int row = first + idx / 16, c = idx % 16;
@@ -378,37 +398,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
         }
         fence_async_smem();
       }
-      tmem_st32(t_s0 + lane_off + sb * 64, pk);
-      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->p_full[sb]);
     }
     if (to) atomicExch(&sh->timed_out, 1);
-
-    // ------------------------------------------------------------------ epilogue
-    const bool have = ntiles > 0 && !to;
-    if (have) {
+    have = __all_sync(0xffffffffu, ntiles > 0 && !to && warp_live);
+    if (ntiles > 0 && !to) {
       if (!mbar_wait(&sh->o_ready[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1)) {
         atomicExch(&sh->timed_out, 1);
+        have = false;
       }
       tc_fence_after();
     }
-    const int64_t orow = (((int64_t)b * (p.M + 1) + gr / p.G) * p.Hq + hq) * 128;
     if (p.nsplit == 1) {
+      // normalised bf16 row -> smem (the Q tile is dead once the last MMA is done),
+      // then the four warps copy whole rows out with coalesced 16-byte stores
       const float inv = (have && valid && l > 0.f) ? 1.f / l : 0.f;
+      uint8_t* ost = q_s;  // [128 rows][256 B], 16-byte chunks rotated by row
+      if (warp_live) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        if (have) {
-          tmem_ld32(t_o + lane_off + c * 32, o);
-          tmem_wait_ld();
-        } else {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          if (have) {
+            tmem_ld32(t_o + lane_off + c * 32, o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
-        }
-        if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + orow + c * 32);
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint4 w;
@@ -416,74 +434,96 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
             w.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
             w.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
             w.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
-            dst[q4] = w;
+            const int chunk = c * 4 + q4;
+            *reinterpret_cast<uint4*>(ost + r * 256 + ((chunk ^ (r & 15)) << 4)) = w;
           }
         }
       }
-    } else {
-      // partial (max, sum, unnormalised O) of this split -> own smem for the cluster merge
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        if (have) {
-          tmem_ld32(t_o + lane_off + c * 32, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
-        }
-        float4* dst = reinterpret_cast<float4*>(o_stage + r * 128 + c * 32);
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          // rotate the 16-byte slots by row to spread shared-memory banks
-          const int slot = (q4 + r) & 7;
-          dst[slot] = make_float4(__uint_as_float(o[4 * slot]), __uint_as_float(o[4 * slot + 1]),
-                                  __uint_as_float(o[4 * slot + 2]), __uint_as_float(o[4 * slot + 3]));
-        }
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+      const int rows = min(kRows, p.rows_total - qtile * kRows);
+      const int t = (warp - 2) * 32 + lane;
+      for (int idx = t; idx < rows * 16; idx += 128) {
+        const int rr = idx >> 4, chunk = idx & 15;
+        const int g2 = qtile * kRows + rr;
+        const int64_t orow = (((int64_t)b * (p.M + 1) + g2 / p.G) * p.Hq + hk * p.G + g2 % p.G) * 128;
+        reinterpret_cast<uint4*>(p.out + orow)[chunk] =
+            *reinterpret_cast<const uint4*>(ost + rr * 256 + ((chunk ^ (rr & 15)) << 4));
       }
-      sh->m_st[r] = have ? m : -INFINITY;
-      sh->l_st[r] = have ? l : 0.f;
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
   if (p.nsplit > 1) {
+    // ---------------------------------------------------------------- split merge
+    // Each split writes (max, sum, O) of its real rows to the workspace (L2),
+    // the cluster barrier orders the writes, and every CTA then merges its
+    // share of the rows from the other splits' records.
     cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
     const int ns = p.nsplit;
+    const int unit = bh * gridDim.y + qtile;
+    // workspace records are chunk-major ([32 float4 chunks][128 rows]) so that a
+    // warp's 32 rows write, and read back, 512 contiguous bytes
+    float4* ws_o = reinterpret_cast<float4*>(p.ws) + (size_t)unit * ns * 32 * kRows;
+    float2* ws_ml = reinterpret_cast<float2*>(p.ws + (size_t)gridDim.z * gridDim.y * ns * kRows * 128) +
+                    (size_t)unit * ns * kRows;
+    if (warp >= 2 && warp_live) {
+      float4* dst = ws_o + (size_t)split * 32 * kRows + r;
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t o[2][32];
+        if (have) {  // warp-uniform: the TMEM reads are warp-collective
+          tmem_ld32(t_o + lane_off + c * 32, o[0]);
+          tmem_ld32(t_o + lane_off + (c + 1) * 32, o[1]);
+          tmem_wait_ld();
+        } else {  // an empty split contributes zeros (its weight is 0 as well)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[0][j] = o[1][j] = 0u;
+        }
+        if (row_ok) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              __stcg(dst + ((c + h) * 8 + q4) * kRows,
+                     make_float4(__uint_as_float(o[h][4 * q4]), __uint_as_float(o[h][4 * q4 + 1]),
+                                 __uint_as_float(o[h][4 * q4 + 2]), __uint_as_float(o[h][4 * q4 + 3])));
+        }
+      }
+      if (row_ok) __stcg(ws_ml + (size_t)split * kRows + r, make_float2(have ? m : -INFINITY, have ? l : 0.f));
+    }
+    __threadfence();
+    tc_fence_before();
+    cluster.sync();  // every split's record is written
     const int rank = (int)cluster.block_rank();
-    const int r_lo = rank * kRows / ns, r_hi = (rank + 1) * kRows / ns;
-    for (int idx = threadIdx.x; idx < (r_hi - r_lo) * 32; idx += blockDim.x) {
-      const int rr = r_lo + idx / 32;
-      const int d = (idx % 32) * 4;
+    const int rows = min(kRows, p.rows_total - qtile * kRows);  // real rows of this tile
+    // rank j merges chunks [q_lo, q_hi) of every real row; consecutive threads take
+    // consecutive rows, so each split's record is read with coalesced loads
+    const int q_lo = rank * 32 / ns, q_hi = (rank + 1) * 32 / ns;
+    for (int idx = threadIdx.x; idx < (q_hi - q_lo) * rows; idx += blockDim.x) {
+      const int rr = idx % rows;
+      const int q = q_lo + idx / rows;
       const int g2 = qtile * kRows + rr;
-      if (g2 >= p.rows_total) continue;
-      float mj[kMaxSplit_tc], lj[kMaxSplit_tc];
+      float2 ml[kMaxSplit_tc];
       float4 oj[kMaxSplit_tc];
 #pragma unroll
       for (int j = 0; j < kMaxSplit_tc; ++j) {
         if (j < ns) {
-          const TcSmem* peer = cluster.map_shared_rank(sh, (unsigned)j);
-          mj[j] = peer->m_st[rr];
-          lj[j] = peer->l_st[rr];
-          oj[j] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(o_stage, (unsigned)j) + rr * 128 + d);
+          ml[j] = __ldcg(ws_ml + (size_t)j * kRows + rr);
+          oj[j] = __ldcg(ws_o + ((size_t)j * 32 + q) * kRows + rr);
         } else {
-          mj[j] = -INFINITY;
-          lj[j] = 0.f;
+          ml[j] = make_float2(-INFINITY, 0.f);
           oj[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
       float mmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kMaxSplit_tc; ++j) mmax = fmaxf(mmax, mj[j]);
+      for (int j = 0; j < kMaxSplit_tc; ++j) mmax = fmaxf(mmax, ml[j].x);
       const float msafe = mmax == -INFINITY ? 0.f : mmax;
       float L = 0.f;
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < kMaxSplit_tc; ++j) {
-        const float w = fast_exp2(mj[j] - msafe);
-        L += w * lj[j];
+        const float w = fast_exp2(ml[j].x - msafe);  // 0 for an empty split
+        L += w * ml[j].y;
         a.x += w * oj[j].x;
         a.y += w * oj[j].y;
         a.z += w * oj[j].z;
@@ -494,9 +534,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
       uint2 pk;
       pk.x = pack_bf16x2(a.x * inv, a.y * inv);
       pk.y = pack_bf16x2(a.z * inv, a.w * inv);
-      *reinterpret_cast<uint2*>(p.out + orow + d) = pk;
+      *reinterpret_cast<uint2*>(p.out + orow + q * 4) = pk;
     }
-    cluster.sync();  // peers may still be reading this CTA's shared memory
+  } else {
+    tc_fence_before();
+    __syncthreads();
   }
   if (warp == 1) {
     tc_fence_after();
@@ -507,31 +549,45 @@ __global__ void __launch_bounds__(kTcThreads, 1) tree_attn_tc_kernel(const __gri
 
 }  // namespace
 
-tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cudaStream_t s) {
+tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& lp) {
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int tiles_q = (p.rows_total + kRows - 1) / kRows;
-  const int64_t units = (int64_t)p.B * p.Hkv * tiles_q;
-  const int key_tiles = (int)std::max<int64_t>(1, (p.S_cap + kKeyTile - 1) / kKeyTile);
+  const int rows_total = (Hq / Hkv) * (M + 1);
+  lp.tiles_q = (rows_total + kRows - 1) / kRows;
+  const int64_t units = (int64_t)B * Hkv * lp.tiles_q;
+  const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
   int ns = (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms + units - 1) / units));
   ns = std::min(ns, key_tiles);
-  p.tiles_per_split = (key_tiles + ns - 1) / ns;
-  p.nsplit = (key_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
-  p.stages = kStages;
-  // At most two CTAs per SM: each holds 256 of the 512 TMEM columns, so an
-  // allocation never waits on a CTA that is itself waiting.
-  const size_t smem = 1024 + kQBytes + (size_t)kStages * kStageBytes + sizeof(TcSmem);
-  e = cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  lp.tiles_per_split = (key_tiles + ns - 1) / ns;
+  lp.nsplit = (key_tiles + lp.tiles_per_split - 1) / lp.tiles_per_split;
+  // Deepest ring that keeps the grid resident: two CTAs per SM when the grid
+  // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
+  // never waits on a CTA that is itself waiting), else one CTA per SM.
+  const int64_t ctas = units * lp.nsplit;
+  const bool two_per_sm = ctas > sms;
+  lp.stages = two_per_sm ? 2 : std::min(kMaxStages, std::max(2, lp.tiles_per_split));
+  const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
+  lp.smem = std::max(smem_min, 1024 + kQBytes + (size_t)lp.stages * kStageBytes + sizeof(TcSmem));
+  lp.ws_bytes = lp.nsplit > 1 ? (size_t)units * lp.nsplit * kRows * (128 + 2) * sizeof(float) : 0;
+  return TV_OK;
+}
+
+tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, const TcPlan& lp,
+                           cudaStream_t s) {
+  p.tiles_per_split = lp.tiles_per_split;
+  p.nsplit = lp.nsplit;
+  p.stages = lp.stages;
+  cudaError_t e = cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
   if (e != cudaSuccess) return record_cuda_error(e);
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tree_attn_tc_kernel, kTcThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tree_attn_tc_kernel, kTcThreads, lp.smem);
   if (e != cudaSuccess) return record_cuda_error(e);
   if (occ > 2 || occ < 1) return TV_ERR_UNSUPPORTED;
-  if ((int64_t)p.B * p.Hkv > 65535 || tiles_q > 65535) return TV_ERR_UNSUPPORTED;
-  dim3 grid(p.nsplit, tiles_q, p.B * p.Hkv);
-  return launch(tree_attn_tc_kernel, grid, dim3(kTcThreads), smem, s, p.nsplit, true, tmk, tmv, p);
+  if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
+  dim3 grid(lp.nsplit, lp.tiles_q, p.B * p.Hkv);
+  return launch(tree_attn_tc_kernel, grid, dim3(kTcThreads), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
 }  // namespace tv

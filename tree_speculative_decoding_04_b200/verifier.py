@@ -52,6 +52,7 @@ class TreeVerifier:
         self.v = v_layers if v_layers is not None else [torch.zeros((B, Hkv, S_cap, D), **bf) for _ in range(L)]
         self.k_ptrs = tv.layer_pointers(self.k, dev)
         self.v_ptrs = tv.layer_pointers(self.v, dev)
+        self.workspace = tv.attention_workspace(B, M, Hq, Hkv, D, S_cap, dev)
         self.logits = torch.zeros((B, self.n, V), dtype=torch.float32, device=dev)
         self.argmax = torch.zeros((B, self.n), **i32)
         self.accept_len = torch.zeros((B,), **i32)
@@ -72,7 +73,7 @@ class TreeVerifier:
 
     def attention(self, layer, stream=None):
         tv.tree_attention(self.q[layer], self.k[layer], self.v[layer], self.kv_start, self.kv_len, self.anc,
-                          self.status, self.out[layer], stream=stream)
+                          self.status, self.out[layer], self.workspace, stream=stream)
 
     def accept(self, stream=None):
         tv.tree_accept(self.logits, self.draft, self.parent, self.depth, self.anc, self.status, self.max_depth,
