@@ -120,6 +120,30 @@ tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v
                          uint16_t* out, void* workspace, size_t workspace_bytes, tv_stream_t stream);
 
 /*
+ * tree_attention_noalloc -- tree_attention for callers that cannot allocate
+ * device memory (for instance a serving process whose memory pool already owns
+ * the whole GPU, or a plugin whose host framework gives it no device
+ * allocator).  The pages have no counterpart: this is a deployment variant.
+ *
+ * Same arguments, layouts and results as tree_attention, without the
+ * workspace: the key-split partials go to a fixed scratch array of
+ * tree_attention_noalloc_max_scratch() bytes (32 MiB) compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  A shape whose tree_attention_workspace_size exceeds that maximum is
+ * rejected with TV_ERR_UNSUPPORTED.  Nothing is allocated: the first call on a
+ * device only looks up the array's device address (make that first call before
+ * any stream capture).  All calls share the one array, so calls that overlap on
+ * the device race with each other; each call overwrites what it reads, so no
+ * clearing is needed between calls.
+ */
+size_t tree_attention_noalloc_max_scratch(void);
+
+tv_status tree_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                                 const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
+                                 int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
+                                 uint16_t* out, tv_stream_t stream);
+
+/*
  * tree_accept -- per-node greedy argmax of the teacher logits fused with
  * longest accepted path selection.  [EAGLE-Pangu, results: accepted length per
  * verification step.]  Node i is accepted iff its parent is accepted and

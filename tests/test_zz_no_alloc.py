@@ -1,0 +1,98 @@
+"""GPU test of tree_attention_noalloc, the allocation-free variant of tree attention.
+
+Some callers cannot allocate device memory -- a serving process whose memory
+pool already owns the whole GPU, or a plugin whose host framework gives it no
+device allocator.  tree_attention_noalloc serves them: the key-split partials go
+to a fixed scratch array inside the library instead of a caller workspace.
+This file checks, through the C ABI, that two calls in a row give the same
+output as tree_attention with a caller-provided workspace (within the attention
+tolerance of the other tests), and that a shape too large for the fixed scratch
+is refused.  It runs last so that a failure here leaves every other test run.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import tree_speculative_decoding_04_b200 as tv
+import workloads as W
+from helpers import assert_attn_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _p(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _inputs(name, seed):
+    cfg = W.CONFIGS[name]
+    dev = torch.device("cuda:0")
+    st = W.make_step(cfg, seed=seed, device=dev, with_logits=False)
+    B, n = cfg.B, cfg.M + 1
+    par = torch.as_tensor(st.parent, device=dev)
+    anc = torch.empty((B, n, (n + 31) // 32), dtype=torch.int32, device=dev)
+    depth = torch.empty((B, n), dtype=torch.int32, device=dev)
+    status = torch.empty((B,), dtype=torch.int32, device=dev)
+    tv.tree_build_mask(par, cfg.max_depth, anc, depth, status)
+    ks = torch.as_tensor(st.kv_start, device=dev)
+    kl = torch.as_tensor(st.kv_len, device=dev)
+    return cfg, st, anc, status, ks, kl
+
+
+def _noalloc(lib, cfg, st, anc, status, ks, kl, out, stream):
+    return lib.tree_attention_noalloc(
+        _p(st.q), _p(st.k), _p(st.v), st.S_cap, _p(ks), _p(kl), _p(anc), _p(status), cfg.B, cfg.M, cfg.Hq,
+        cfg.Hkv, cfg.D, ctypes.c_float(cfg.D ** -0.5), _p(out), ctypes.c_void_p(stream))
+
+
+def _with_workspace(lib, cfg, st, anc, status, ks, kl, out, stream):
+    nbytes = lib.tree_attention_workspace_size(cfg.B, cfg.M, cfg.Hq, cfg.Hkv, cfg.D, st.S_cap)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=out.device)
+    rc = lib.tree_attention(
+        _p(st.q), _p(st.k), _p(st.v), st.S_cap, _p(ks), _p(kl), _p(anc), _p(status), cfg.B, cfg.M, cfg.Hq,
+        cfg.Hkv, cfg.D, ctypes.c_float(cfg.D ** -0.5), _p(out), _p(ws), nbytes, ctypes.c_void_p(stream))
+    return rc, ws
+
+
+def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
+    lib = tv.load()
+    cap = lib.tree_attention_noalloc_max_scratch()
+    first = _inputs("mha7b", seed=3)
+    second = _inputs("eqspec", seed=4)
+    for cfg, st, *_ in (first, second):
+        need = lib.tree_attention_workspace_size(cfg.B, cfg.M, cfg.Hq, cfg.Hkv, cfg.D, st.S_cap)
+        assert 0 < need <= cap  # both shapes go through the scratch array
+    stream = torch.cuda.current_stream().cuda_stream
+    outs = []
+    # two calls in a row, no synchronisation in between: the second reuses the scratch
+    for cfg, st, anc, status, ks, kl in (first, second):
+        out = torch.full_like(st.q, float("nan"))
+        assert _noalloc(lib, cfg, st, anc, status, ks, kl, out, stream) == 0
+        outs.append(out)
+    torch.cuda.synchronize()
+    for (cfg, st, anc, status, ks, kl), got in zip((first, second), outs):
+        ref = torch.full_like(st.q, float("nan"))
+        rc, ws = _with_workspace(lib, cfg, st, anc, status, ks, kl, ref, stream)
+        assert rc == 0
+        torch.cuda.synchronize()
+        g = got.float().cpu().numpy()
+        r = ref.float().cpu().numpy()
+        assert np.isfinite(g).all()
+        assert_attn_close(g, r, f"noalloc vs workspace ({cfg.name})")
+
+
+def test_noalloc_refuses_shapes_beyond_its_scratch():
+    lib = tv.load()
+    cap = lib.tree_attention_noalloc_max_scratch()
+    M, Hq, Hkv, D, S_cap = 16, 1, 1, 128, 4096
+    # a batch just below two CTAs per SM still splits every sequence's keys in two
+    sizes = {B: lib.tree_attention_workspace_size(B, M, Hq, Hkv, D, S_cap) for B in range(2, 600)}
+    B = max(sizes, key=sizes.get)
+    need = sizes[B]
+    assert need > cap
+    dummy = ctypes.c_void_p(256)  # never touched: the call must refuse on the host
+    rc = lib.tree_attention_noalloc(dummy, dummy, dummy, S_cap, dummy, dummy, dummy, dummy, B, M, Hq, Hkv, D,
+                                    ctypes.c_float(0.088), dummy, ctypes.c_void_p(0))
+    assert rc == 2  # TV_ERR_UNSUPPORTED

@@ -26,6 +26,8 @@ EXPORTS = (
     "tree_build_mask",
     "tree_attention_workspace_size",
     "tree_attention",
+    "tree_attention_noalloc_max_scratch",
+    "tree_attention_noalloc",
     "tree_accept",
     "kv_commit_realign",
     "tv_status_string",
@@ -54,6 +56,10 @@ def load(path: str = LIB_PATH):
     lib.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
     lib.tree_attention_workspace_size.restype = ctypes.c_size_t
     lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, ctypes.c_size_t, P]
+    lib.tree_attention_noalloc_max_scratch.argtypes = []
+    lib.tree_attention_noalloc_max_scratch.restype = ctypes.c_size_t
+    lib.tree_attention_noalloc.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
+    lib.tree_attention_noalloc.restype = ctypes.c_int
     lib.tree_accept.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, P]
     lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P]
     for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign"):

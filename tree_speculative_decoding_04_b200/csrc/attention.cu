@@ -481,3 +481,94 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
   }
   return run_attention_tc(tmk, tmv, p, plan, s);
 }
+
+// ---------------------------------------------------------------------------
+// tree_attention_noalloc: the same computation for callers that cannot
+// allocate device memory -- for example a serving process whose memory pool
+// already owns the whole GPU, or a plugin whose host framework hands it no
+// device allocator.  The split partials then live in a fixed array compiled
+// into this library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace tv {
+namespace {
+
+// 32 MiB of scratch; every GPU that loads this library holds it until the
+// process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name only stands in for it, so the address is looked up once per
+// device, with that device current, and cached.
+tv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (dev < 0 || dev >= kMaxDevices) return TV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return TV_OK;
+}
+
+}  // namespace
+}  // namespace tv
+
+extern "C" size_t tree_attention_noalloc_max_scratch(void) { return tv::kNoAllocScratchBytes; }
+
+extern "C" tv_status tree_attention_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                            int64_t S_cap, const int32_t* kv_start, const int32_t* kv_len,
+                                            const uint32_t* anc_mask, int32_t* status, int B, int M, int Hq,
+                                            int Hkv, int D, float scale, uint16_t* out, tv_stream_t stream) {
+  using namespace tv;
+  if (B < 0 || M < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || !(scale > 0.f)) return TV_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return TV_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
+  if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
+  if (B == 0) return TV_OK;
+  if (!q || !k || !v || !kv_start || !kv_len || !anc_mask || !status || !out) return TV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TV_ERR_INVALID_ARG;
+  AttnParams p;
+  p.q = q;
+  p.kv_start = kv_start;
+  p.kv_len = kv_len;
+  p.anc = anc_mask;
+  p.status = status;
+  p.out = out;
+  p.S_cap = S_cap;
+  p.B = B;
+  p.M = M;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.W = (M + 1 + 31) / 32;
+  p.rows_total = p.G * (M + 1);
+  p.nsplit = p.tiles_per_split = p.stages = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.ws = nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap tmk, tmv;
+  if (!encode_kv_map(&tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&tmv, v, B * Hkv, S_cap, D))
+    return TV_ERR_INVALID_ARG;
+  if (D == 64) return run<64>(tmk, tmv, p, s);  // this path keeps its partials on chip
+  TcPlan plan;
+  tv_status r = plan_attention_tc(B, M, Hq, Hkv, S_cap, plan);
+  if (r != TV_OK) return r;
+  if (plan.ws_bytes > 0) {
+    if (plan.ws_bytes > kNoAllocScratchBytes) return TV_ERR_UNSUPPORTED;  // shape too large for the fixed scratch
+    void* scratch = nullptr;
+    r = noalloc_scratch(&scratch);
+    if (r != TV_OK) return r;
+    p.ws = static_cast<float*>(scratch);
+  }
+  return run_attention_tc(tmk, tmv, p, plan, s);
+}
