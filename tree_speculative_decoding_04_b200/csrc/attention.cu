@@ -463,7 +463,7 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
   p.G = Hq / Hkv;
   p.W = (M + 1 + 31) / 32;
   p.rows_total = p.G * (M + 1);
-  p.nsplit = p.tiles_per_split = p.stages = 0;
+  p.nsplit = p.tiles_per_split = p.stages = p.v_stages = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.ws = nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -552,7 +552,7 @@ extern "C" tv_status tree_attention_noalloc(const uint16_t* q, const uint16_t* k
   p.G = Hq / Hkv;
   p.W = (M + 1 + 31) / 32;
   p.rows_total = p.G * (M + 1);
-  p.nsplit = p.tiles_per_split = p.stages = 0;
+  p.nsplit = p.tiles_per_split = p.stages = p.v_stages = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.ws = nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

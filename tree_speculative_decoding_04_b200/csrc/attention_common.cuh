@@ -23,7 +23,8 @@ struct AttnParams {
   int rows_total;       // G * (M + 1) query rows per (sequence, kv head)
   int nsplit;           // key splits (cluster size along x)
   int tiles_per_split;  // 64-key tiles per split
-  int stages;
+  int stages;           // key-tile ring depth (K ring of the tensor-core kernel)
+  int v_stages;         // V ring depth of the tensor-core kernel
   float scale_log2;     // softmax scale * log2(e)
   float* ws;            // split partials: [units][nsplit][128 rows][128] O, then [units][nsplit][128][2] (m, l)
 };
@@ -62,7 +63,7 @@ inline bool encode_kv_map(CUtensorMap* map, const void* base, int BH, int64_t S_
 
 // Tensor-core (tcgen05) path for head dim 128; defined in attention_tc.cu.
 struct TcPlan {
-  int tiles_q, nsplit, tiles_per_split, stages;
+  int tiles_q, nsplit, tiles_per_split, stages, v_stages;
   size_t smem, ws_bytes;
 };
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& plan);

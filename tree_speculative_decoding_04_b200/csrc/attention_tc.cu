@@ -7,10 +7,14 @@
 // applied from the ancestor bitmask on the last M+1 key columns only.
 //
 // One CTA owns 128 query rows (tree node x q head of one GQA group) of one
-// (sequence, kv head) and one split of the key range; the splits of a query
-// tile form a thread-block cluster and merge through distributed shared memory.
+// (sequence, kv head) and one split of that sequence's key range.  The splits
+// of a query tile form a thread-block cluster: each writes its partial (max,
+// sum, O) to a workspace in L2, the cluster barrier orders the writes, and each
+// CTA then merges 1/nsplit of the output columns.
 // Warp roles (192 threads):
-//   warp 0      TMA producer: 64-key K and V tiles into a 2-stage smem ring
+//   warp 0      TMA producer: 64-key K tiles and V tiles into two separate smem
+//               rings -- a K slot is freed as soon as S = QK^T has read it, a V
+//               slot only after O += PV, so the V ring is the deeper one
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_i = Q K_i^T   (M=128, N=64, K=128; A, B from smem)   -> TMEM S[i%2]
 //                 O  += P_i V_i   (M=128, N=128, K=64; A=P from TMEM, B=V from smem) -> TMEM O
@@ -39,7 +43,6 @@ constexpr int kTmemCols = 256;
 constexpr int kMaxStages = 6;
 constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
 constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
-constexpr int kStageBytes = 2 * kTileBytes;
 constexpr float kRescaleThreshold = 8.0f;        // log2 domain
 constexpr int kMaxSplit_tc = 8;                  // portable cluster size
 
@@ -123,8 +126,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) 
 }
 
 struct TcSmem {
-  uint64_t kv_full[kMaxStages];
-  uint64_t kv_empty[kMaxStages];
+  uint64_t k_full[kMaxStages];
+  uint64_t k_empty[kMaxStages];
+  uint64_t v_full[kMaxStages];
+  uint64_t v_empty[kMaxStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_ready[2];  // PV_j completes a phase of o_ready[j % 2]
@@ -150,18 +155,19 @@ __device__ __forceinline__ uint64_t anc_window(const uint32_t (&aw)[kMaxRows / 3
 
 // O += P_j V_j for key tile j (one thread), then release the K/V stage and
 // publish the new O.  Returns false if P_j never arrived.
-__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t t_s0, uint32_t t_o, int j,
-                                         int stages) {
+__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t t_s0, uint32_t t_o, int j,
+                                         int v_stages) {
   const uint32_t idesc_o = idesc_bf16(128, 128, 1);
-  const int sb = j & 1, s = j % stages;
+  const int sb = j & 1, s = j % v_stages;
   if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1)) return false;
+  if (!mbar_wait(&sh->v_full[s], (j / v_stages) & 1)) return false;
   tc_fence_after();
-  const uint32_t v_addr = smem_u32(stage_s + s * kStageBytes + kTileBytes);
+  const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
 #pragma unroll
   for (int kk = 0; kk < kKeyTile / 16; ++kk)
     mma_ts(t_o, t_s0 + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
            (j > 0 || kk > 0) ? 1u : 0u);
-  tc_commit(&sh->kv_empty[s]);
+  tc_commit(&sh->v_empty[s]);
   tc_commit(&sh->o_ready[j & 1]);
   return true;
 }
@@ -169,12 +175,17 @@ __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* stage_s, uint32_t 
 __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                                                                     const __grid_constant__ CUtensorMap tmv,
                                                                     const __grid_constant__ AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The 128-byte-swizzled tiles need 1024-byte alignment.  The dynamic window
+  // starts on such a boundary on this GPU; if it ever did not, every CTA treats
+  // its sequence as failed (zero output, TV_SEQ_TIMEOUT) instead of computing.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  const bool aligned_ok = (smem_u32(smem_raw) & 1023u) == 0;
   uint8_t* q_s = smem;                              // [2][128][128 B]
-  const int stages = p.stages;
-  uint8_t* stage_s = smem + kQBytes;                // [stages][K box0, K box1, V box0, V box1]
-  TcSmem* sh = reinterpret_cast<TcSmem*>(stage_s + stages * kStageBytes);
+  const int k_stages = p.stages, v_stages = p.v_stages;
+  uint8_t* k_ring = smem + kQBytes;                   // [k_stages][2 boxes of 64 rows x 128 B]
+  uint8_t* v_ring = k_ring + k_stages * kTileBytes;   // [v_stages][2 boxes]
+  TcSmem* sh = reinterpret_cast<TcSmem*>(v_ring + v_stages * kTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -186,9 +197,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
 
   if (threadIdx.x == 0) {
     sh->timed_out = 0;
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&sh->kv_full[s], 1);
-      mbar_init(&sh->kv_empty[s], 1);
+    for (int s = 0; s < k_stages; ++s) {
+      mbar_init(&sh->k_full[s], 1);
+      mbar_init(&sh->k_empty[s], 1);
+    }
+    for (int s = 0; s < v_stages; ++s) {
+      mbar_init(&sh->v_full[s], 1);
+      mbar_init(&sh->v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sh->s_full[s], 1);
@@ -207,27 +222,37 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   pdl_launch_dependents();
   const int32_t ks = p.kv_start[b];
   const int32_t kl = p.kv_len[b];
-  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const bool valid = aligned_ok && p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
   const int N = kl + p.M + 1;
-  const int t0 = split * p.tiles_per_split;
-  const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + kKeyTile - 1) / kKeyTile - t0)) : 0;
+  // this sequence's key tiles are dealt evenly over the splits (ragged batches
+  // would otherwise leave short sequences in one split)
+  const int seq_tiles = (N + kKeyTile - 1) / kKeyTile;
+  const int tps = (seq_tiles + p.nsplit - 1) / p.nsplit;
+  const int t0 = split * tps;
+  const int ntiles = valid ? max(0, min(tps, seq_tiles - t0)) : 0;
   const int k_lo = t0 * kKeyTile;
 
   // The first ring's worth of K/V tiles and the Q tile are requested before the
   // TMEM allocation barrier, so their memory latency overlaps the set-up.
-  auto issue_kv = [&](int i) {
-    const int s = i % stages;
-    mbar_arrive_expect_tx(&sh->kv_full[s], kStageBytes);
-    const int col = ks + k_lo + i * kKeyTile;
-    uint8_t* st = stage_s + s * kStageBytes;
-    tma_load_3d(st, &tmk, &sh->kv_full[s], 0, col, bh);
-    tma_load_3d(st + kBoxBytes, &tmk, &sh->kv_full[s], 64, col, bh);
-    tma_load_3d(st + kTileBytes, &tmv, &sh->kv_full[s], 0, col, bh);
-    tma_load_3d(st + kTileBytes + kBoxBytes, &tmv, &sh->kv_full[s], 64, col, bh);
+  auto issue_k = [&](int i) {
+    const int s = i % k_stages;
+    uint8_t* dst = k_ring + s * kTileBytes;
+    mbar_arrive_expect_tx(&sh->k_full[s], kTileBytes);
+    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks + k_lo + i * kKeyTile, bh);
+    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks + k_lo + i * kKeyTile, bh);
   };
-  const int prologue_tiles = min(ntiles, stages);
+  auto issue_v = [&](int i) {
+    const int s = i % v_stages;
+    uint8_t* dst = v_ring + s * kTileBytes;
+    mbar_arrive_expect_tx(&sh->v_full[s], kTileBytes);
+    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks + k_lo + i * kKeyTile, bh);
+    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks + k_lo + i * kKeyTile, bh);
+  };
   if (warp == 0 && lane == 0)  // the thread that initialised the barriers
-    for (int i = 0; i < prologue_tiles; ++i) issue_kv(i);
+    for (int i = 0; i < min(ntiles, max(k_stages, v_stages)); ++i) {
+      if (i < k_stages) issue_k(i);
+      if (i < v_stages) issue_v(i);
+    }
   const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
   const int gr = qtile * kRows + r;
   const bool row_ok = gr < p.rows_total;
@@ -261,21 +286,35 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // K_i waits for S_{i-k_stages} to finish, V_i for PV_{i-v_stages}; both
+      // complete in the order this loop issues, so it never blocks early
       bool to = false;
-      int issued = prologue_tiles;
-      for (int i = prologue_tiles; i < ntiles && !to; ++i) {
-        const int s = i % stages;
-        if (!mbar_wait(&sh->kv_empty[s], ((i / stages) - 1) & 1)) {
-          to = true;
-          break;
+      int k_issued = min(ntiles, k_stages), v_issued = min(ntiles, v_stages);
+      for (int i = 0; i < ntiles && !to; ++i) {
+        if (i >= k_stages) {
+          if (!mbar_wait(&sh->k_empty[i % k_stages], ((i / k_stages) - 1) & 1)) {
+            to = true;
+            break;
+          }
+          issue_k(i);
+          ++k_issued;
         }
-        issue_kv(i);
-        ++issued;
+        if (i >= v_stages) {
+          if (!mbar_wait(&sh->v_empty[i % v_stages], ((i / v_stages) - 1) & 1)) {
+            to = true;
+            break;
+          }
+          issue_v(i);
+          ++v_issued;
+        }
       }
       if (to) {
         atomicExch(&sh->timed_out, 1);
         // copies still in flight must land before this CTA's shared memory is released
-        for (int i = max(0, issued - stages); i < issued; ++i) mbar_wait(&sh->kv_full[i % stages], (i / stages) & 1);
+        for (int i = max(0, k_issued - k_stages); i < k_issued; ++i)
+          mbar_wait(&sh->k_full[i % k_stages], (i / k_stages) & 1);
+        for (int i = max(0, v_issued - v_stages); i < v_issued; ++i)
+          mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -285,23 +324,24 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       const uint32_t q_addr = smem_u32(q_s);
       bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
-        const int s = i % stages, sb = i & 1;
-        if (!mbar_wait(&sh->kv_full[s], (i / stages) & 1)) {
+        const int s = i % k_stages, sb = i & 1;
+        if (!mbar_wait(&sh->k_full[s], (i / k_stages) & 1)) {
           to = true;
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(stage_s + s * kStageBytes);
+        const uint32_t k_addr = smem_u32(k_ring + s * kTileBytes);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
           const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
           mma_ss(t_s0 + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
         }
+        tc_commit(&sh->k_empty[s]);
         tc_commit(&sh->s_full[sb]);
-        if (i >= 1 && !issue_pv(sh, stage_s, t_s0, t_o, i - 1, stages)) to = true;
+        if (i >= 1 && !issue_pv(sh, v_ring, t_s0, t_o, i - 1, v_stages)) to = true;
       }
-      if (!to && !issue_pv(sh, stage_s, t_s0, t_o, ntiles - 1, stages)) to = true;
+      if (!to && !issue_pv(sh, v_ring, t_s0, t_o, ntiles - 1, v_stages)) to = true;
       if (to) {
         atomicExch(&sh->timed_out, 1);
         // let every MMA issued so far retire before TMEM and shared memory are released
@@ -333,9 +373,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         tmem_ld32(t_s0 + lane_off + sb * 64, sr[0]);
         tmem_ld32(t_s0 + lane_off + sb * 64 + 32, sr[1]);
         tmem_wait_ld();
-        float x[64];
+        float x[64];  // raw scores; the scale is folded into the exponent's FFMA
 #pragma unroll
-        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sr[j >> 5][j & 31]) * p.scale_log2;
+        for (int j = 0; j < 64; ++j) x[j] = __uint_as_float(sr[j >> 5][j & 31]);
         if (key0 + kKeyTile > kl) {  // tile reaches the tree rows or the end of the range
           const int np = kl - key0;  // prefix keys in this tile
           const uint64_t pre = np >= 64 ? ~0ull : (np <= 0 ? 0ull : ((1ull << np) - 1ull));
@@ -349,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(fmaxf(fmaxf(x[q], x[q + 8]), fmaxf(x[q + 16], x[q + 24])),
                                                   fmaxf(fmaxf(x[q + 32], x[q + 40]), fmaxf(x[q + 48], x[q + 56])));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
         if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
           if (m != -INFINITY) {
             // O holds earlier tiles: rescale this row once PV_{i-1} has landed
@@ -378,7 +418,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = fast_exp2(x[2 * j] - ms), p1 = fast_exp2(x[2 * j + 1] - ms);
+          const float p0 = fast_exp2(fmaf(x[2 * j], p.scale_log2, -ms));
+          const float p1 = fast_exp2(fmaf(x[2 * j + 1], p.scale_log2, -ms));
           rs8[j & 7] += p0 + p1;
           pk[j] = pack_bf16x2(p0, p1);
         }
@@ -389,7 +430,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       // past the end of the key range the V rows may hold anything: zero them
       const int kend = N - key0;
       if (kend < kKeyTile) {
-        uint8_t* vt = stage_s + (i % stages) * kStageBytes + kTileBytes;
+        uint8_t* vt = v_ring + (i % v_stages) * kTileBytes;
+        if (!mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1)) to = true;  // V_i must have landed
         const int first = max(kend, 0);
         for (int idx = r; idx < (kKeyTile - first) * 16; idx += kRows) {
           const int row = first + idx / 16, c = idx % 16;
@@ -544,7 +586,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && sh->timed_out) atomicOr(&p.status[b], kSeqTimeout);
+  if (threadIdx.x == 0 && (sh->timed_out || !aligned_ok)) atomicOr(&p.status[b], kSeqTimeout);
 }
 
 }  // namespace
@@ -567,9 +609,12 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   // never waits on a CTA that is itself waiting), else one CTA per SM.
   const int64_t ctas = units * lp.nsplit;
   const bool two_per_sm = ctas > sms;
-  lp.stages = two_per_sm ? 2 : std::min(kMaxStages, std::max(2, lp.tiles_per_split));
+  // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
+  // one CTA per SM: K ring 3, V ring up to 6
+  lp.stages = two_per_sm ? 2 : std::min(3, std::max(2, lp.tiles_per_split));
+  lp.v_stages = two_per_sm ? 3 : std::min(kMaxStages, std::max(2, lp.tiles_per_split));
   const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
-  lp.smem = std::max(smem_min, 1024 + kQBytes + (size_t)lp.stages * kStageBytes + sizeof(TcSmem));
+  lp.smem = std::max(smem_min, kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem));
   lp.ws_bytes = lp.nsplit > 1 ? (size_t)units * lp.nsplit * kRows * (128 + 2) * sizeof(float) : 0;
   return TV_OK;
 }
@@ -579,6 +624,7 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   p.tiles_per_split = lp.tiles_per_split;
   p.nsplit = lp.nsplit;
   p.stages = lp.stages;
+  p.v_stages = lp.v_stages;
   cudaError_t e = cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
   if (e != cudaSuccess) return record_cuda_error(e);
   int occ = 0;
