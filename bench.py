@@ -80,6 +80,8 @@ def barrier(world):
 
 
 def max_over_ranks(x, world, device):
+    """The largest x over all ranks (device: where the reduction tensor lives --
+    the rank's GPU under NCCL, the CPU under gloo)."""
     if world == 1:
         return x
     import torch.distributed as dist
@@ -87,6 +89,20 @@ def max_over_ranks(x, world, device):
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank, ms_total_max, steps):
+    """Units per second over all ranks: every rank did the same work, the job
+    took as long as the slowest rank."""
+    return world * units_per_rank / (ms_total_max / steps * 1e-3)
+
+
+def config_dict(cfg, world, kv_len):
+    return {"workload": f"{cfg.name}: {W.describe(cfg)}", "global_batch": cfg.B * world,
+            "prefix": cfg.prefix, "tree_rows": cfg.M + 1, "layers": cfg.L, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: every step streams %.2f GB of distinct per-layer KV" %
+                  (cfg.L * attention_bytes(cfg, kv_len) / 1e9),
+            "timing": "CUDA graph of one step replayed K times; CUDA events on the launching stream"}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -329,7 +345,7 @@ def run_reference(args, cfg, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {W.describe(cfg)}"},
+        "config": config_dict(cfg, world, host["kv_len"]),
         "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -338,12 +354,28 @@ def run_reference(args, cfg, world, rank):
 
 # ----------------------------------------------------------------------------- our arm
 
+def physical_layers(cfg, device):
+    """Layers of KV cache that fit in 60% of the free device memory (all of them
+    for every workload except the 80-layer ragged stress case)."""
+    P = W.make_prefix_lengths(cfg, np.random.default_rng(0))
+    _, _, S_cap = W.cache_geometry(cfg, P)
+    per_layer = 2 * cfg.B * cfg.Hkv * S_cap * cfg.D * 2
+    free, _ = torch.cuda.mem_get_info(device)
+    return max(1, min(cfg.L, int(0.6 * free // per_layer)))
+
+
 def run_ours(args, cfg, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     import tree_speculative_decoding_04_b200 as tvpkg
 
     tvpkg.load()
+    L_cfg = cfg.L
+    L_phys = physical_layers(cfg, device)
+    if L_phys < cfg.L:
+        import dataclasses
+
+        cfg = dataclasses.replace(cfg, L=L_phys)
     ver, host = build_workload(cfg, args.seed, device)
     stream = torch.cuda.Stream(device)
     ks0 = ver.kv_start.clone()
@@ -382,7 +414,7 @@ def run_ours(args, cfg, world, rank, local):
     barrier(world)
     ms_total = max_over_ranks(e0.elapsed_time(e1), world, device)
     ms_step = ms_total / args.steps
-    value = world * cfg.B * cfg.M / (ms_step * 1e-3)
+    value = whole_job_rate(world, cfg.B * cfg.M, ms_total, args.steps)
 
     # ---- results of one step (for the algorithmic byte counts)
     with torch.cuda.stream(stream):
@@ -459,7 +491,7 @@ def run_ours(args, cfg, world, rank, local):
         cpu = {"value": cfg.B * cfg.M / t_step, "unit": "nodes/s", "cores": 1, "kind": "oracle", "sample": desc,
                "host_threads_available": os.cpu_count()}
     return finish(args, cfg, world, rank, value, ms_step, roofline, kv_commit, mask_ms, attn_ms, attn_single_ms,
-                  acc_ms, com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device)
+                  acc_ms, com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device, L_cfg)
 
 
 def run_e2e(args, cfg, ver, host, reset, stream, world, device):
@@ -501,7 +533,7 @@ def run_e2e(args, cfg, ver, host, reset, stream, world, device):
 
 
 def finish(args, cfg, world, rank, value, ms_step, roofline, kv_commit, mask_ms, attn_ms, attn_single_ms, acc_ms,
-           com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device):
+           com_ms, reset_ms, al, cpu, e2e, ver, clk, kl_h, device, L_cfg):
     L = cfg.L
     if rank != 0:
         return
@@ -510,11 +542,8 @@ def finish(args, cfg, world, rank, value, ms_step, roofline, kv_commit, mask_ms,
         "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: {W.describe(cfg)}", "global_batch": cfg.B * world,
-                   "prefix": cfg.prefix, "tree_rows": cfg.M + 1, "layers": cfg.L, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: every step streams %.2f GB of distinct per-layer KV" %
-                         (cfg.L * attention_bytes(cfg, kl_h) / 1e9),
-                   "timing": "CUDA graph of one step replayed K times; CUDA events on the launching stream"},
+        "config": dict(config_dict(cfg, world, kl_h), layers_in_workload=L_cfg,
+                       layers_measured=cfg.L),
         "roofline": roofline,
         "kv_commit": kv_commit,
         "breakdown_us": {"tree_build_mask": mask_ms * 1e3, "tree_attention_per_layer": attn_ms * 1e3,
