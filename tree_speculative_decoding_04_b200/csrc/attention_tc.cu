@@ -600,7 +600,9 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   lp.tiles_q = (rows_total + kRows - 1) / kRows;
   const int64_t units = (int64_t)B * Hkv * lp.tiles_q;
   const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
-  int ns = (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms + units - 1) / units));
+  // Split the key range only while the query tiles alone leave SMs idle: a
+  // split adds a merge, and past one CTA per SM it adds a partial second wave.
+  int ns = units >= sms ? 1 : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms + units - 1) / units));
   ns = std::min(ns, key_tiles);
   lp.tiles_per_split = (key_tiles + ns - 1) / ns;
   lp.nsplit = (key_tiles + lp.tiles_per_split - 1) / lp.tiles_per_split;

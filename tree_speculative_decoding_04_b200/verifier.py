@@ -65,7 +65,8 @@ class TreeVerifier:
 
     # ------------------------------------------------------------------ device path
     def launches_per_step(self) -> int:
-        """Kernels this library launches per step (mask 1, attention L, accept 2, commit 2)."""
+        """Kernels this library launches per step: mask 1, attention 1 per layer,
+        accept 2, commit 2."""
         return 1 + self.L + 2 + 2
 
     def build_mask(self, stream=None):
