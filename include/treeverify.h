@@ -130,7 +130,9 @@ tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v
  * tree_attention_noalloc_max_scratch() bytes (32 MiB) compiled into the
  * library, which every GPU that loads the library holds until the process
  * exits.  A shape whose tree_attention_workspace_size exceeds that maximum is
- * rejected with TV_ERR_UNSUPPORTED.  Nothing is allocated: the first call on a
+ * rejected with TV_ERR_UNSUPPORTED; on a 148-SM GPU none does (the key split
+ * stops once the query tiles fill the SMs, so the partials stay below about
+ * 3 x 148 x 66,560 bytes).  Nothing is allocated: the first call on a
  * device only looks up the array's device address (make that first call before
  * any stream capture).  All calls share the one array, so calls that overlap on
  * the device race with each other; each call overwrites what it reads, so no

@@ -6,8 +6,8 @@ device allocator.  tree_attention_noalloc serves them: the key-split partials go
 to a fixed scratch array inside the library instead of a caller workspace.
 This file checks, through the C ABI, that two calls in a row give the same
 output as tree_attention with a caller-provided workspace (within the attention
-tolerance of the other tests), and that a shape too large for the fixed scratch
-is refused.  It runs last so that a failure here leaves every other test run.
+tolerance of the other tests), and that every split plan of this GPU fits the
+fixed scratch.  It runs last so that a failure here leaves every other test run.
 """
 import ctypes
 
@@ -83,16 +83,20 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls():
         assert_attn_close(g, r, f"noalloc vs workspace ({cfg.name})")
 
 
-def test_noalloc_refuses_shapes_beyond_its_scratch():
+def test_noalloc_scratch_holds_every_split_plan():
+    """The key-split plan stops splitting once the query tiles alone fill the
+    SMs, so its partials never exceed about 3 x SMs x 128 rows x 130 floats
+    (about 29.6 MB on 148 SMs): on this GPU every shape that tree_attention
+    serves fits the fixed scratch, and the size check that refuses larger
+    workspaces is never reached."""
     lib = tv.load()
     cap = lib.tree_attention_noalloc_max_scratch()
-    M, Hq, Hkv, D, S_cap = 16, 1, 1, 128, 4096
-    # a batch just below two CTAs per SM still splits every sequence's keys in two
-    sizes = {B: lib.tree_attention_workspace_size(B, M, Hq, Hkv, D, S_cap) for B in range(2, 600)}
-    B = max(sizes, key=sizes.get)
-    need = sizes[B]
-    assert need > cap
-    dummy = ctypes.c_void_p(256)  # never touched: the call must refuse on the host
-    rc = lib.tree_attention_noalloc(dummy, dummy, dummy, S_cap, dummy, dummy, dummy, dummy, B, M, Hq, Hkv, D,
-                                    ctypes.c_float(0.088), dummy, ctypes.c_void_p(0))
-    assert rc == 2  # TV_ERR_UNSUPPORTED
+    worst = 0
+    for Hq, Hkv in ((1, 1), (8, 8), (32, 32), (32, 8), (28, 4), (64, 8)):
+        for M in (3, 16, 63, 127, 255):
+            for S_cap in (64, 4096, 65536):
+                for B in range(1, 301):
+                    need = lib.tree_attention_workspace_size(B, M, Hq, Hkv, 128, S_cap)
+                    assert need <= cap, (B, M, Hq, Hkv, S_cap, need, cap)
+                    worst = max(worst, need)
+    assert worst > cap // 2  # the sweep reaches the plans that split the most

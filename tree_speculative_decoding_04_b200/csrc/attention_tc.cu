@@ -532,7 +532,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       }
       if (row_ok) __stcg(ws_ml + (size_t)split * kRows + r, make_float2(have ? m : -INFINITY, have ? l : 0.f));
     }
-    __threadfence();
+    // barrier.cluster.arrive releases and barrier.cluster.wait acquires at
+    // cluster scope, which orders the records' global stores for every CTA of
+    // the cluster: no separate device-scope fence is needed
     tc_fence_before();
     cluster.sync();  // every split's record is written
     const int rank = (int)cluster.block_rank();
@@ -602,7 +604,7 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
   // Split the key range only while the query tiles alone leave SMs idle: a
   // split adds a merge, and past one CTA per SM it adds a partial second wave.
-  int ns = units >= sms ? 1 : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms + units - 1) / units));
+  int ns = units >= sms ? 1 : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms) / units));
   ns = std::min(ns, key_tiles);
   lp.tiles_per_split = (key_tiles + ns - 1) / ns;
   lp.nsplit = (key_tiles + lp.tiles_per_split - 1) / lp.tiles_per_split;
