@@ -384,12 +384,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
           for (int j = 0; j < 64; ++j)
             if (!((allowed >> j) & 1ull)) x[j] = -INFINITY;
         }
-        float mx8[8];
+        // row maximum: four chains of three-input maxima over the 64 scores
+        float c4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = fmaxf(fmaxf(fmaxf(x[q], x[q + 8]), fmaxf(x[q + 16], x[q + 24])),
-                                                  fmaxf(fmaxf(x[q + 32], x[q + 40]), fmaxf(x[q + 48], x[q + 56])));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * p.scale_log2;
+        for (int q = 0; q < 30; ++q) c4[q & 3] = fmax3(c4[q & 3], x[4 + 2 * q], x[5 + 2 * q]);
+        const float mx = fmaxf(fmax3(c4[0], c4[1], c4[2]), c4[3]) * p.scale_log2;
         if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
           if (m != -INFINITY) {
             // O holds earlier tiles: rescale this row once PV_{i-1} has landed
@@ -414,16 +413,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
           m = mx;
         }
         const float ms = m == -INFINITY ? 0.f : m;
+        // exponent argument and row sum two keys at a time (packed FP32 pairs)
         uint32_t pk[32];
-        float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(-ms, -ms);
+        uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float p0 = fast_exp2(fmaf(x[2 * j], p.scale_log2, -ms));
-          const float p1 = fast_exp2(fmaf(x[2 * j + 1], p.scale_log2, -ms));
-          rs8[j & 7] += p0 + p1;
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), sc2, nm2), a0, a1);
+          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          rs2[j & 3] = f2_add(rs2[j & 3], f2_pack(p0, p1));
           pk[j] = pack_bf16x2(p0, p1);
         }
-        l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        {
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(rs2[0], s0, s1);
+          f2_unpack(rs2[1], s2, s3);
+          f2_unpack(rs2[2], s4, s5);
+          f2_unpack(rs2[3], s6, s7);
+          l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        }
         tmem_st32(t_s0 + lane_off + sb * 64, pk);
         tmem_wait_st();
       }
