@@ -37,7 +37,10 @@ import workloads as W  # noqa: E402
 METRIC = "verified tree nodes/sec + KV-commit GB/s on 1 B200; fraction of roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
-ATTN_SRC = os.path.join(ROOT, "tree_speculative_decoding_04_b200", "csrc", "attention.cu")
+# the sources of the tensor-core attention kernel: its traffic figure holds only
+# for the exact sources it was measured on
+ATTN_SRCS = [os.path.join(ROOT, "tree_speculative_decoding_04_b200", "csrc", f)
+             for f in ("attention_tc.cu", "attention_common.cuh", "tv_common.cuh", "attention.cu")]
 
 
 def parse():
@@ -241,13 +244,21 @@ def capture(fn, stream):
     return g
 
 
+def attention_source_sha256():
+    h = hashlib.sha256()
+    for path in ATTN_SRCS:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def read_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, only if the
     kernel source has not changed since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
-        sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+        sha = attention_source_sha256()
         if rec.get("source_sha256") == sha:
             return rec
     except Exception:

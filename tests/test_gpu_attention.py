@@ -67,6 +67,7 @@ def _inputs(B, M, Hq, Hkv, D, P, seed, left_padded=False, tree="uniform", max_de
         (2, 33, 8, 1, 128, 500),  # MQA, two mask words
         (1, 255, 2, 1, 128, 200),  # largest tree
         (4, 20, 12, 4, 128, [64, 65, 127, 129]),  # tile edges
+        (2, 85, 6, 2, 128, [70, 300]),  # 258 query rows: three query tiles, the last with 2 rows
     ],
 )
 def test_parity_full(orc, B, M, Hq, Hkv, D, P):
