@@ -252,14 +252,15 @@ def attention_source_sha256():
     return h.hexdigest()
 
 
-def read_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, only if the
-    kernel source has not changed since the counters were taken."""
+def read_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, only for the
+    workload it was captured on and only if the kernel sources have not changed
+    since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
         sha = attention_source_sha256()
-        if rec.get("source_sha256") == sha:
+        if rec.get("source_sha256") == sha and rec.get("workload") == workload:
             return rec
     except Exception:
         pass
@@ -477,9 +478,9 @@ def run_ours(args, cfg, world, rank, local):
     a_bytes = attention_bytes(cfg, kl_h)
     a_flops = attention_flops(cfg, kl_h, depth)
     achieved = a_bytes / (attn_ms * 1e-3) / 1e9
-    traffic = read_traffic()
+    traffic = read_traffic(cfg.name)
     roofline = {
-        "bound": "hbm", "kernel": "tree_attn_kernel", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+        "bound": "hbm", "kernel": "tree_attn_tc_kernel" if cfg.D == 128 else "tree_attn_mma_kernel", "achieved": achieved, "peak": hbm, "unit": "GB/s",
         "frac": achieved / hbm, "peak_kind": f"{peak_kind} copy bandwidth (burst)",
         "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
         "algorithmic_bytes_per_launch": a_bytes, "launch_us": attn_ms * 1e3,
