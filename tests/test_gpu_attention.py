@@ -116,6 +116,29 @@ def test_no_leak_between_branches(orc, P):
         np.testing.assert_array_equal(o[0, u], base[0, u])
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_single_row_maximum_jumps(orc, D):
+    """A key that only one query row scores highly, far into the prefix: that row's
+    running maximum jumps by far more than the lazy-rescale threshold while the
+    other rows of its warp keep theirs, so the O rescale runs for some rows of a
+    warp and not for others (it must stay warp-collective)."""
+    B, M, Hq, Hkv = 1, 63, 2, 1
+    P = 1000
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, P, seed=21)
+    spikes = [(5, 0, 700, 3), (40, 1, 300, 17), (63, 0, 900, 40)]  # (row, q-head, key, channel)
+    for u, h, key, ch in spikes:
+        q[0, :, :, ch] = 0.0  # only the spiking row sees the spike key's channel
+    for u, h, key, ch in spikes:
+        q[0, u, h, ch] = 1.0
+        k[0, 0, key, :] = 0.0
+        k[0, 0, key, ch] = 16.0 * D ** 0.5  # score 16 / ln 2 = 23 in the log2 domain
+    got, ref, _ = _run(orc, q, k, v, par, ks, kl)
+    assert np.isfinite(got).all()
+    assert_attn_close(got, ref, "attention with single-row maximum jumps")
+    for u, h, key, ch in spikes:  # the spiking row is (almost) the spike key's value row
+        np.testing.assert_allclose(got[0, u, h], v[0, 0, key].float().cpu().numpy(), atol=2e-2, rtol=2e-2)
+
+
 def test_invalid_sequences_zero_rows(orc):
     B, M, Hq, Hkv, D = 4, 10, 8, 4, 128
     q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, 300, seed=2)

@@ -174,7 +174,8 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(co
     const uint32_t sbase = smem_u32(smem);
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % stages;
-      if (!mbar_wait(&full[s], (i / stages) & 1)) {
+      // decided for the whole warp: the ldmatrix / mma.sync below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / stages) & 1))) {
         atomicExch(&timed_out, 1);
         break;
       }

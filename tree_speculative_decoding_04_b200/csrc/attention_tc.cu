@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       anc_w[w] = w < p.W ? __ldg(p.anc + ((int64_t)b * (p.M + 1) + u) * p.W + w) : 0u;
   }
   if (warp == 1) {
+    __syncwarp();  // tcgen05.alloc is warp-collective
     tmem_alloc(&sh->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -360,7 +361,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     bool to = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1;
-      if (!mbar_wait(&sh->s_full[sb], (i >> 1) & 1)) {
+      // every wait that gates a TMEM access is decided for the whole warp: the
+      // tcgen05.ld / tcgen05.st that follow are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (i >> 1) & 1))) {
         to = true;
         break;
       }
@@ -389,29 +392,35 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
 #pragma unroll
         for (int q = 0; q < 30; ++q) c4[q & 3] = fmax3(c4[q & 3], x[4 + 2 * q], x[5 + 2 * q]);
         const float mx = fmaxf(fmax3(c4[0], c4[1], c4[2]), c4[3]) * p.scale_log2;
-        if (mx > m + kRescaleThreshold) {  // also true on the first finite tile (m = -inf)
-          if (m != -INFINITY) {
-            // O holds earlier tiles: rescale this row once PV_{i-1} has landed
-            const float corr = fast_exp2(m - mx);
-            if (!mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1)) {
-              to = true;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld32(t_o + lane_off + c * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
-              tmem_st32(t_o + lane_off + c * 32, o);
-            }
-            tmem_wait_st();
-            l *= corr;
+        // Lazy rescale: a row moves its reference maximum only when the tile's
+        // maximum exceeds it by more than the threshold (always on its first
+        // finite tile, where m = -inf).  Rescaling O is a TMEM access, which is
+        // warp-collective, so the warp rescales when any of its rows needs it,
+        // each row by its own factor (1 for a row whose maximum stays, and for
+        // a row with no finite score yet, whose O row is still zero).
+        const bool grow = mx > m + kRescaleThreshold;
+        const bool scale_o = grow && m != -INFINITY;
+        if (__any_sync(0xffffffffu, scale_o)) {
+          // O holds earlier tiles: rescale once PV_{i-1} has landed
+          if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1))) {
+            to = true;
+            break;
           }
-          m = mx;
+          tc_fence_after();
+          const float corr = scale_o ? fast_exp2(m - mx) : 1.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(t_o + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+            tmem_st32(t_o + lane_off + c * 32, o);
+          }
+          tmem_wait_st();
+          l *= corr;
         }
+        if (grow) m = mx;
         const float ms = m == -INFINITY ? 0.f : m;
         // exponent argument and row sum two keys at a time (packed FP32 pairs)
         uint32_t pk[32];
@@ -440,7 +449,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       const int kend = N - key0;
       if (kend < kKeyTile) {
         uint8_t* vt = v_ring + (i % v_stages) * kTileBytes;
-        if (!mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1)) to = true;  // V_i must have landed
+        if (!__all_sync(0xffffffffu, mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1)))
+          to = true;  // V_i must have landed
         const int first = max(kend, 0);
         for (int idx = r; idx < (kKeyTile - first) * 16; idx += kRows) {
           const int row = first + idx / 16, c = idx % 16;
@@ -462,6 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       }
       tc_fence_after();
     }
+    have = __all_sync(0xffffffffu, have);  // gates warp-collective TMEM reads
     if (p.nsplit == 1) {
       // normalised bf16 row -> smem (the Q tile is dead once the last MMA is done),
       // then the four warps copy whole rows out with coalesced 16-byte stores
@@ -594,6 +605,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     __syncthreads();
   }
   if (warp == 1) {
+    __syncwarp();  // tcgen05.dealloc is warp-collective
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
