@@ -518,11 +518,10 @@ def run_e2e(args, cfg, ver, host, reset, stream, world, device):
             c0 = int(host["kv_start"][b] + host["kv_len"][b])
             h["tree_k"][layer, b].copy_(ver.k[layer][b, :, c0:c0 + cfg.M + 1].cpu())
             h["tree_v"][layer, b].copy_(ver.v[layer][b, :, c0:c0 + cfg.M + 1].cpu())
-    geom = (host["kv_start"].tolist(), host["kv_len"].tolist())
 
     def e2e_step():
         reset()
-        ver.step_from_host(h, geometry=geom, stream=stream)
+        ver.step_from_host(h, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(max(1, args.warmup // 2)):

@@ -199,6 +199,29 @@ tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers
                             int32_t* kv_start, int32_t* kv_len, int32_t* max_len, int realign,
                             uint8_t* attn_mask, int32_t* pos_ids, tv_stream_t stream);
 
+/*
+ * tree_kv_write -- place the K and V rows of the current step's M+1 tree nodes
+ * behind each sequence's committed prefix, in every layer: the cache layout
+ * that tree_attention and kv_commit_realign read.  The pages have no separate
+ * step for it (their branch caches are written by the model's own forward);
+ * it is the append that this library's cache layout needs, offered so that a
+ * caller holding the new rows in one staging buffer needs no per-sequence
+ * copies and no host copy of the geometry.
+ *
+ *   k_layers, v_layers  DEVICE arrays of L device pointers to bf16
+ *             [B][Hkv][S_cap][D] layers (16-byte aligned), written
+ *   tree_k, tree_v  bf16 [L][B][Hkv][M+1][D] in (16-byte aligned)
+ *   kv_start, kv_len  int32 [B] in: row r of sequence b goes to column
+ *             kv_start[b] + kv_len[b] + r
+ *   D in {64, 128}; 0 <= M < 256.
+ * A sequence whose geometry breaks 0 <= kv_start, 0 <= kv_len,
+ * kv_start + kv_len + M + 1 <= S_cap is left untouched (tree_attention then
+ * gives it zero rows and kv_commit_realign flags it TV_SEQ_BAD_GEOMETRY).
+ */
+tv_status tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, const uint16_t* tree_k,
+                        const uint16_t* tree_v, int L, int B, int Hkv, int D, int64_t S_cap, int M,
+                        const int32_t* kv_start, const int32_t* kv_len, tv_stream_t stream);
+
 /* Human-readable name of a tv_status. */
 const char* tv_status_string(tv_status s);
 

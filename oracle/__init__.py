@@ -55,6 +55,7 @@ def lib():
         _lib.oracle_argmax_rows.argtypes = [P, i64, i32, P]
         _lib.oracle_tree_accept.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P]
         _lib.oracle_kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P]
+        _lib.oracle_tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P]
         for f in (
             _lib.oracle_tree_build_mask,
             _lib.oracle_tree_attention_rows,
@@ -196,3 +197,23 @@ def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_
     if with_status:
         return ks, kl, int(ml[0]), am, pos, st
     return ks, kl, int(ml[0]), am, pos
+
+
+def tree_kv_write(k_layers, v_layers, tree_k, tree_v, kv_start, kv_len):
+    """In place on the uint16 arrays in k_layers / v_layers (each [B][Hkv][S_cap][D]):
+    tree_k / tree_v uint16 [L][B][Hkv][M+1][D] go to columns kv_start + kv_len + r."""
+    L = len(k_layers)
+    assert L == len(v_layers) and L >= 1
+    B, Hkv, S_cap, D = k_layers[0].shape
+    for a in list(k_layers) + list(v_layers):
+        assert a.dtype == np.uint16 and a.flags.c_contiguous and a.shape == (B, Hkv, S_cap, D)
+    tk, tv = _c(tree_k, np.uint16), _c(tree_v, np.uint16)
+    assert tk.shape == tv.shape and tk.shape[:3] == (L, B, Hkv) and tk.shape[4] == D
+    M = tk.shape[3] - 1
+    kp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in k_layers])
+    vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_layers])
+    ks, kl = _c(kv_start, np.int32), _c(kv_len, np.int32)  # kept alive across the call
+    rc = lib().oracle_tree_kv_write(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), _p(tk),
+                                    _p(tv), L, B, Hkv, D, S_cap, M, _p(ks), _p(kl))
+    if rc:
+        raise ValueError("oracle_tree_kv_write rc=%d" % rc)

@@ -391,3 +391,32 @@ int oracle_kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layer
   free(nb);
   return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Appending the step's tree rows to the cache.
+ * [EP] 2.C evaluates all speculative tokens in one teacher pass against the
+ * cached prefix; in this layout the M+1 tree rows of sequence b sit right
+ * behind its prefix, row r at column kv_start[b] + kv_len[b] + r, in every
+ * layer.  tree_k / tree_v are [L][B][Hkv][M+1][D]; a sequence whose rows would
+ * not fit the cache (or whose geometry is negative) is left untouched.
+ * ------------------------------------------------------------------------- */
+int oracle_tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, const uint16_t* tree_k,
+                         const uint16_t* tree_v, int L, int B, int Hkv, int D, int64_t S_cap, int M,
+                         const int32_t* kv_start, const int32_t* kv_len) {
+  const int n = M + 1;
+  for (int l = 0; l < L; ++l)
+    for (int b = 0; b < B; ++b) {
+      if (!geometry_ok(kv_start[b], kv_len[b], M, S_cap)) continue;
+      for (int h = 0; h < Hkv; ++h)
+        for (int r = 0; r < n; ++r) {
+          const int64_t src = ((((int64_t)l * B + b) * Hkv + h) * n + r) * D;
+          const int64_t col = (int64_t)kv_start[b] + kv_len[b] + r;
+          const int64_t dst = (((int64_t)b * Hkv + h) * S_cap + col) * D;
+          for (int d = 0; d < D; ++d) {
+            k_layers[l][dst + d] = tree_k[src + d];
+            v_layers[l][dst + d] = tree_v[src + d];
+          }
+        }
+    }
+  return 0;
+}

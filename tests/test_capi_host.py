@@ -77,6 +77,13 @@ def test_argument_errors_are_synchronous(lib):
                                  z, z, z) == 1
     assert lib.kv_commit_realign(dummy, dummy, 1, 1, 1, 80, 64, 3, dummy, dummy, dummy, 3, dummy, dummy, dummy, 0,
                                  z, z, z) == 2
+    # tree-row append: negative size, unsupported D, tree too large, null rows, misaligned rows, empty
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, -1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 96, 64, 3, dummy, dummy, z) == 2
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 128, 512, 256, dummy, dummy, z) == 2
+    assert lib.tree_kv_write(dummy, dummy, z, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
+    assert lib.tree_kv_write(dummy, dummy, P(264), dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
+    assert lib.tree_kv_write(z, z, z, z, 0, 1, 1, 128, 64, 3, z, z, z) == 0
 
 
 def test_binding_refuses_host_tensors():

@@ -23,4 +23,5 @@ from ._lib import (  # noqa: F401
     tree_attention,
     tree_attention_workspace_size,
     tree_build_mask,
+    tree_kv_write,
 )

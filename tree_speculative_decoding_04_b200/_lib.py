@@ -30,6 +30,7 @@ EXPORTS = (
     "tree_attention_noalloc",
     "tree_accept",
     "kv_commit_realign",
+    "tree_kv_write",
     "tv_status_string",
     "tv_last_cuda_error",
     "tv_version",
@@ -62,7 +63,8 @@ def load(path: str = LIB_PATH):
     lib.tree_attention_noalloc.restype = ctypes.c_int
     lib.tree_accept.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, P]
     lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P]
-    for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign"):
+    lib.tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P]
+    for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign", "tree_kv_write"):
         getattr(lib, name).restype = ctypes.c_int
     lib.tv_status_string.argtypes = [ctypes.c_int]
     lib.tv_status_string.restype = ctypes.c_char_p
@@ -188,6 +190,22 @@ def kv_commit_realign(k_layer_ptrs, v_layer_ptrs, B, Hkv, D, S_cap, M, path, acc
                                   _ptr(accept_len), _ptr(status), int(max_depth), _ptr(kv_start), _ptr(kv_len),
                                   _ptr(max_len), int(realign), _ptr(attn_mask), _ptr(pos_ids), _stream(stream))
     _check(rc, "kv_commit_realign")
+
+
+def tree_kv_write(k_layer_ptrs, v_layer_ptrs, tree_k, tree_v, S_cap, kv_start, kv_len, stream=None):
+    """tree_k / tree_v bf16 [L][B][Hkv][M+1][D] -> the cache of every layer, at
+    columns kv_start + kv_len + r (k_layer_ptrs / v_layer_ptrs as for
+    kv_commit_realign)."""
+    L, B, Hkv, n, D = tree_k.shape
+    _need(k_layer_ptrs, torch.int64, (L,), "k_layer_ptrs")
+    _need(v_layer_ptrs, torch.int64, (L,), "v_layer_ptrs")
+    _need(tree_k, torch.bfloat16, (L, B, Hkv, n, D), "tree_k")
+    _need(tree_v, torch.bfloat16, (L, B, Hkv, n, D), "tree_v")
+    _need(kv_start, torch.int32, (B,), "kv_start")
+    _need(kv_len, torch.int32, (B,), "kv_len")
+    rc = load().tree_kv_write(_ptr(k_layer_ptrs), _ptr(v_layer_ptrs), _ptr(tree_k), _ptr(tree_v), L, B, Hkv, D,
+                              int(S_cap), n - 1, _ptr(kv_start), _ptr(kv_len), _stream(stream))
+    _check(rc, "tree_kv_write")
 
 
 def layer_pointers(layers, device=None) -> torch.Tensor:
