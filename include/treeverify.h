@@ -36,9 +36,10 @@
  *     0 <= parent[i] < i.
  *   - bf16 tensors are passed as uint16_t bit patterns.
  *   - KV cache of one layer: [B][Hkv][S_cap][D] bf16.  Sequence b's committed
- *     prefix is columns [kv_start[b], kv_start[b] + kv_len[b]); the caller has
- *     written the M+1 tree rows of the current step right behind it, at columns
- *     kv_start[b] + kv_len[b] + r, r = 0..M.  A sequence whose geometry breaks
+ *     prefix is columns [kv_start[b], kv_start[b] + kv_len[b]); the M+1 tree
+ *     rows of the current step sit right behind it, at columns
+ *     kv_start[b] + kv_len[b] + r, r = 0..M (written by the caller, or by
+ *     tree_kv_write from a [L][B][Hkv][M+1][D] staging buffer).  A sequence whose geometry breaks
  *     0 <= kv_start, 0 <= kv_len, kv_start + kv_len + M + 1 <= S_cap is flagged
  *     TV_SEQ_BAD_GEOMETRY and skipped.
  */
