@@ -44,6 +44,7 @@ constexpr int kMaxStages = 6;
 constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
 constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
 constexpr float kRescaleThreshold = 8.0f;        // log2 domain
+constexpr int kPrefetchTiles = 1;                 // key tiles per CTA warmed in L2 before the grid dependency
 constexpr int kMaxSplit_tc = 8;                  // portable cluster size
 
 // ------------------------------------------------------------------ tcgen05 wrappers
@@ -217,6 +218,36 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
+  }
+  // With programmatic launch this CTA can be resident while the previous kernel
+  // is still finishing.  Until the grid dependency resolves, warm L2 with the
+  // first key tiles of this split and with this CTA's query rows.  A prefetch
+  // binds no value: a write of the previous kernel to the same lines lands in
+  // L2, which every later read goes through, so a stale geometry read here only
+  // wastes the prefetch (issued only for a geometry that fits the cache, so the
+  // coordinates stay inside the tensor).
+  if (warp == 0 && lane == 0) {
+    const int32_t ks_h = __ldcg(p.kv_start + b), kl_h = __ldcg(p.kv_len + b);
+    if (geometry_ok(ks_h, kl_h, p.M, p.S_cap)) {
+      const int st = (kl_h + p.M + 1 + kKeyTile - 1) / kKeyTile;
+      const int tp = (st + p.nsplit - 1) / p.nsplit;
+      const int nt = min(kPrefetchTiles, max(0, min(tp, st - split * tp)));
+      for (int i = 0; i < nt; ++i) {
+        const int row = ks_h + (split * tp + i) * kKeyTile;
+        tma_prefetch_3d(&tmk, 0, row, bh);
+        tma_prefetch_3d(&tmk, 64, row, bh);
+        tma_prefetch_3d(&tmv, 0, row, bh);
+        tma_prefetch_3d(&tmv, 64, row, bh);
+      }
+    }
+  }
+  if (warp >= 2) {
+    const int gr_h = qtile * kRows + (warp & 3) * 32 + lane;
+    if (gr_h < p.rows_total) {
+      const uint16_t* qr = p.q + (((int64_t)b * (p.M + 1) + gr_h / p.G) * p.Hq + hk * p.G + gr_h % p.G) * 128;
+      prefetch_l2(qr);
+      prefetch_l2(qr + 64);
+    }
   }
   pdl_wait_primary();
   pdl_launch_dependents();
