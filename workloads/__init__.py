@@ -63,6 +63,11 @@ CONFIGS = {
                      logit_sigma=2.0, left_padded=True),
 }
 
+# The eqspec shapes in per-sequence-length mode (every sequence's content starts
+# at column 0, no padding): the commit appends in place and nothing is realigned,
+# which is what cross-batch grouping of equal lengths buys a padded batch.
+CONFIGS["eqspec_ragged"] = dataclasses.replace(CONFIGS["eqspec"], name="eqspec_ragged", left_padded=False)
+
 CONFIG_ORDER = ["tiny", "mha7b", "eqspec", "b32gqa", "stress"]
 
 
