@@ -267,6 +267,27 @@ def read_traffic(workload):
     return None
 
 
+def roofline_entry(a_bytes, a_flops, attn_ms, hbm, tflops, peak_kind, traffic, kernel):
+    """Roofline of one attention launch: roofline time = max(bytes / bandwidth,
+    flops / tensor peak); the larger term names the bound, and achieved / peak
+    are given in that term's unit."""
+    attn_s = attn_ms * 1e-3
+    tensor_bound = a_flops / (tflops * 1e12) > a_bytes / (hbm * 1e9)
+    r = {
+        "bound": "tensor" if tensor_bound else "hbm",
+        "kernel": kernel,
+        "achieved": a_flops / attn_s / 1e12 if tensor_bound else a_bytes / attn_s / 1e9,
+        "peak": tflops if tensor_bound else hbm,
+        "unit": "TFLOP/s" if tensor_bound else "GB/s",
+        "peak_kind": f"{peak_kind} sustained bf16 GEMM" if tensor_bound else f"{peak_kind} copy bandwidth",
+        "traffic": traffic,
+        "algorithmic_bytes_per_launch": a_bytes, "algorithmic_flops_per_launch": a_flops, "launch_us": attn_ms * 1e3,
+        "hbm_gbs": a_bytes / attn_s / 1e9, "tensor_tflops": a_flops / attn_s / 1e12,
+    }
+    r["frac"] = r["achieved"] / r["peak"]
+    return r
+
+
 def peaks():
     """(HBM copy GB/s, sustained bf16 TFLOP/s, "measured" | "fallback").  The
     attention launches are timed inside a long step, so a tensor-bound launch is
@@ -480,23 +501,10 @@ def run_ours(args, cfg, world, rank, local):
     hbm, tflops, peak_kind = peaks()
     a_bytes = attention_bytes(cfg, kl_h)
     a_flops = attention_flops(cfg, kl_h, depth)
-    attn_s = attn_ms * 1e-3
     traffic = read_traffic(cfg.name)
-    # roofline time = max(bytes / bandwidth, flops / tensor peak); the larger term
-    # names the bound the launch is held to
-    tensor_bound = a_flops / (tflops * 1e12) > a_bytes / (hbm * 1e9)
-    roofline = {
-        "bound": "tensor" if tensor_bound else "hbm",
-        "kernel": "tree_attn_tc_kernel" if cfg.D == 128 else "tree_attn_mma_kernel",
-        "achieved": a_flops / attn_s / 1e12 if tensor_bound else a_bytes / attn_s / 1e9,
-        "peak": tflops if tensor_bound else hbm,
-        "unit": "TFLOP/s" if tensor_bound else "GB/s",
-        "peak_kind": f"{peak_kind} sustained bf16 GEMM" if tensor_bound else f"{peak_kind} copy bandwidth",
-        "traffic": (traffic["dram_bytes_per_launch"] if traffic else None),
-        "algorithmic_bytes_per_launch": a_bytes, "algorithmic_flops_per_launch": a_flops, "launch_us": attn_ms * 1e3,
-        "hbm_gbs": a_bytes / attn_s / 1e9, "tensor_tflops": a_flops / attn_s / 1e12,
-    }
-    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    roofline = roofline_entry(a_bytes, a_flops, attn_ms, hbm, tflops, peak_kind,
+                              traffic["dram_bytes_per_launch"] if traffic else None,
+                              "tree_attn_tc_kernel" if cfg.D == 128 else "tree_attn_mma_kernel")
     c_bytes = commit_bytes(cfg, path, al, kl_h, cfg.left_padded, shift)
     kv_commit = {"gbs": c_bytes / (com_ms * 1e-3) / 1e9, "bytes_per_step": c_bytes, "us": com_ms * 1e3,
                  "frac_hbm": c_bytes / (com_ms * 1e-3) / 1e9 / hbm}
