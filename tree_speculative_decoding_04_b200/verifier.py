@@ -197,7 +197,8 @@ class TreeVerifier:
         layer's tree rows are written into the cache and its attention runs as
         soon as that layer's section has landed; accept_len / path / bonus come
         back into the pinned result buffers.  Asynchronous: synchronise on
-        `stream` before reading the results."""
+        `stream` before reading the results, and before rewriting the staging
+        buffer for the next step (its copies may still be in flight)."""
         h = host if host is not None else self.pinned_inputs()
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         if self._copy_stream is None:
