@@ -93,3 +93,18 @@ def test_binding_refuses_host_tensors():
     with pytest.raises(tv.TVError):
         tv.tree_build_mask(parent, 3, torch.zeros((1, 4, 1), dtype=torch.int32),
                            torch.zeros((1, 4), dtype=torch.int32), torch.zeros((1,), dtype=torch.int32))
+
+
+def test_status_bits_agree_between_header_binding_and_oracle():
+    """The per-sequence status bits carry the same meaning in the header, the
+    binding and the oracle (defined separately in each: no shared source)."""
+    import oracle
+
+    txt = open(os.path.join(ROOT, "include", "treeverify.h")).read()
+    hdr = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define TV_(SEQ_\w+|MAX_TREE_ROWS)\s+(\d+)", txt)}
+    assert hdr == {"SEQ_BAD_PARENT": 1, "SEQ_TOO_DEEP": 2, "SEQ_TIMEOUT": 4, "SEQ_BAD_GEOMETRY": 8,
+                   "MAX_TREE_ROWS": 256}
+    for name, val in hdr.items():
+        assert getattr(tv, name) == val
+    assert (oracle.BAD_PARENT, oracle.TOO_DEEP, oracle.BAD_GEOMETRY) == (
+        hdr["SEQ_BAD_PARENT"], hdr["SEQ_TOO_DEEP"], hdr["SEQ_BAD_GEOMETRY"])
