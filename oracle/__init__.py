@@ -29,33 +29,62 @@ TOO_DEEP = 2
 BAD_GEOMETRY = 8
 
 
-def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so next to it (gcc, -O2, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
+_LIB_OMP = os.path.join(_HERE, "liboracle_omp.so")
+
+
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, no fast-math).
+    openmp=True builds the same source with -fopenmp into liboracle_omp.so: the
+    loops over independent output rows then run on every host core (the
+    arithmetic of each row is unchanged).  Only the benchmark's CPU arms use it."""
+    out = _LIB_OMP if openmp else _LIB
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + ".tmp%d" % os.getpid()
+        extra = ["-fopenmp"] if openmp else []
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math"] + extra + ["-o", tmp, _SRC, "-lm"]
         )
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, out)
+    return out
 
 
 _lib = None
+_use_openmp = False
+
+
+def use_openmp(on: bool = True) -> None:
+    """Select the all-cores build for every later call (must be chosen before
+    the first call; the benchmark's CPU arms only)."""
+    global _use_openmp
+    if _lib is not None and bool(on) != _use_openmp:
+        raise RuntimeError("oracle library already loaded")
+    _use_openmp = bool(on)
+
+
+def threads() -> int:
+    """Host threads the loaded oracle build uses (1 unless the all-cores build is in use)."""
+    if not _use_openmp:
+        return 1
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
 
 
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = ctypes.CDLL(build(openmp=_use_openmp))
         P = ctypes.c_void_p
         i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         _lib.oracle_tree_build_mask.argtypes = [P, i32, i32, i32, P, P, P]
-        _lib.oracle_tree_attention_rows.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, P, i64, P]
-        _lib.oracle_tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, P]
+        _lib.oracle_tree_attention_rows.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, f64, P,
+                                                    i64, P]
+        _lib.oracle_tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f64, f64, P]
         _lib.oracle_argmax_rows.argtypes = [P, i64, i32, P]
         _lib.oracle_tree_accept.argtypes = [P, P, P, P, i32, i32, i32, i32, P, P, P, P]
         _lib.oracle_kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P]
-        _lib.oracle_tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P]
+        _lib.oracle_tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P, f64]
+        _lib.oracle_rope_rows.argtypes = [P, P, i64, i32, f64]
+        _lib.oracle_round_bf16.argtypes = [P, i64, P]
         for f in (
             _lib.oracle_tree_build_mask,
             _lib.oracle_tree_attention_rows,
@@ -102,8 +131,10 @@ def tree_build_mask(parent: np.ndarray, max_depth: int):
     return anc, depth, status
 
 
-def tree_attention(q, k, v, kv_start, kv_len, parent, status, Hkv: int, scale: float | None = None):
-    """q bf16-bits [B][M+1][Hq][D]; k, v bf16-bits [B][Hkv][S_cap][D] -> float64 [B][M+1][Hq][D]."""
+def tree_attention(q, k, v, kv_start, kv_len, parent, status, Hkv: int, scale: float | None = None,
+                   rope_base: float = 0.0):
+    """q bf16-bits [B][M+1][Hq][D]; k, v bf16-bits [B][Hkv][S_cap][D] -> float64 [B][M+1][Hq][D].
+    rope_base > 0: each query row is first rotated to position kv_len + depth(u)."""
     q, k, v = _bits16(q), _bits16(k), _bits16(v)
     B, n, Hq, D = q.shape
     S_cap = k.shape[2]
@@ -114,14 +145,16 @@ def tree_attention(q, k, v, kv_start, kv_len, parent, status, Hkv: int, scale: f
         scale = 1.0 / math.sqrt(D)
     out = np.zeros((B, n, Hq, D), np.float64)
     rc = lib().oracle_tree_attention(
-        _p(q), _p(k), _p(v), S_cap, _p(ks), _p(kl), _p(par), _p(st), B, n - 1, Hq, Hkv, D, scale, _p(out)
+        _p(q), _p(k), _p(v), S_cap, _p(ks), _p(kl), _p(par), _p(st), B, n - 1, Hq, Hkv, D, scale,
+        float(rope_base), _p(out)
     )
     if rc:
         raise ValueError("oracle_tree_attention rc=%d" % rc)
     return out
 
 
-def tree_attention_rows(q, k, v, kv_start, kv_len, parent, status, Hkv: int, sel, scale: float | None = None):
+def tree_attention_rows(q, k, v, kv_start, kv_len, parent, status, Hkv: int, sel, scale: float | None = None,
+                        rope_base: float = 0.0):
     """Only the rows listed in sel ([n][3] of (b, u, q_head)) -> float64 [n][D]."""
     q, k, v = _bits16(q), _bits16(k), _bits16(v)
     B, n, Hq, D = q.shape
@@ -134,7 +167,7 @@ def tree_attention_rows(q, k, v, kv_start, kv_len, parent, status, Hkv: int, sel
     out = np.zeros((sel.shape[0], D), np.float64)
     rc = lib().oracle_tree_attention_rows(
         _p(q), _p(k), _p(v), S_cap, _p(ks), _p(kl), _p(par), _p(st), B, n - 1, Hq, Hkv, D, scale,
-        _p(sel), sel.shape[0], _p(out),
+        float(rope_base), _p(sel), sel.shape[0], _p(out),
     )
     if rc:
         raise ValueError("oracle_tree_attention_rows rc=%d" % rc)
@@ -199,9 +232,11 @@ def kv_commit_realign(k_layers, v_layers, M: int, path, accept_len, status, max_
     return ks, kl, int(ml[0]), am, pos
 
 
-def tree_kv_write(k_layers, v_layers, tree_k, tree_v, kv_start, kv_len):
+def tree_kv_write(k_layers, v_layers, tree_k, tree_v, kv_start, kv_len, depth=None, rope_base: float = 0.0):
     """In place on the uint16 arrays in k_layers / v_layers (each [B][Hkv][S_cap][D]):
-    tree_k / tree_v uint16 [L][B][Hkv][M+1][D] go to columns kv_start + kv_len + r."""
+    tree_k / tree_v uint16 [L][B][Hkv][M+1][D] go to columns kv_start + kv_len + r.
+    depth [B][M+1] with rope_base > 0: K rows are rotated to position kv_len + depth
+    and stored as the nearest bf16."""
     L = len(k_layers)
     assert L == len(v_layers) and L >= 1
     B, Hkv, S_cap, D = k_layers[0].shape
@@ -213,7 +248,30 @@ def tree_kv_write(k_layers, v_layers, tree_k, tree_v, kv_start, kv_len):
     kp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in k_layers])
     vp = (ctypes.c_void_p * L)(*[a.ctypes.data for a in v_layers])
     ks, kl = _c(kv_start, np.int32), _c(kv_len, np.int32)  # kept alive across the call
+    dep = None if depth is None else _c(depth, np.int32)
     rc = lib().oracle_tree_kv_write(ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), _p(tk),
-                                    _p(tv), L, B, Hkv, D, S_cap, M, _p(ks), _p(kl))
+                                    _p(tv), L, B, Hkv, D, S_cap, M, _p(ks), _p(kl),
+                                    None if dep is None else _p(dep), float(rope_base))
     if rc:
         raise ValueError("oracle_tree_kv_write rc=%d" % rc)
+
+
+def rope_rows(x, pos, base: float):
+    """Rotary embedding: rows x [n][D] (float64) rotated by the angles of their
+    positions pos [n]; returns a new array."""
+    x = np.array(x, np.float64, copy=True, order="C")
+    n, D = x.shape
+    pos = _c(pos, np.float64)
+    assert pos.shape == (n,)
+    rc = lib().oracle_rope_rows(_p(x), _p(pos), n, D, float(base))
+    if rc:
+        raise ValueError("oracle_rope_rows rc=%d" % rc)
+    return x
+
+
+def round_bf16(x):
+    """Nearest bf16 (ties to even) of each float64, as uint16 bits."""
+    x = _c(x, np.float64)
+    out = np.zeros(x.shape, np.uint16)
+    lib().oracle_round_bf16(_p(x), x.size, _p(out))
+    return out

@@ -118,15 +118,68 @@ static int geometry_ok(int32_t ks, int32_t kl, int M, int64_t S_cap) {
   return ks >= 0 && kl >= 0 && (int64_t)ks + kl + M + 1 <= S_cap;
 }
 
+/* ---------------------------------------------------------------------------
+ * Rotary position embedding of the tree rows.
+ * [BSD] 2, position-ID contiguity: position IDs run from 0 without gaps over the
+ * attended columns (the condition a rotary embedding needs).  Reading adopted
+ * for a tree: the committed prefix holds positions 0 .. kv_len-1 and node u sits
+ * at position kv_len + depth(u), so every root-to-node path continues the prefix
+ * without a gap (siblings share a position).  The rotation is the published
+ * rotary embedding (RoFormer, Su et al.) in the half-split arrangement: the pair
+ * (x[i], x[i + D/2]), i < D/2, is turned by the angle pos * base^(-2i/D).
+ * ------------------------------------------------------------------------- */
+static void rope_rotate(double* x, int D, double pos, double base) {
+  const int h = D / 2;
+  for (int i = 0; i < h; ++i) {
+    const double th = pos * pow(base, -2.0 * i / D);
+    const double c = cos(th), s = sin(th);
+    const double a = x[i], b = x[i + h];
+    x[i] = a * c - b * s;
+    x[i + h] = b * c + a * s;
+  }
+}
+
+/* rows x [rows][D] rotated in place, row i by the angle set of position pos[i]. */
+int oracle_rope_rows(double* x, const double* pos, int64_t rows, int D, double base) {
+  if (D <= 0 || D % 2 != 0 || !(base > 0.0)) return -1;
+  for (int64_t i = 0; i < rows; ++i) rope_rotate(x + i * D, D, pos[i], base);
+  return 0;
+}
+
+/* Round a double to the nearest bf16 (ties to even), in one rounding: scale the
+ * significand to 8 bits, round it with rint (round-to-nearest-even mode), scale
+ * back; 8 significant bits are exact in a float, whose upper 16 bits are the
+ * bf16 pattern.  Finite values of ordinary range only (no subnormal care). */
+static uint16_t double_to_bf16(double v) {
+  if (v != v) return 0x7FC0;
+  if (v == 0.0) return signbit(v) ? 0x8000 : 0;
+  int e;
+  const double m = frexp(v, &e); /* v = m * 2^e, 0.5 <= |m| < 1 */
+  const double r = ldexp(rint(ldexp(m, 8)), e - 8);
+  const float f = (float)r;
+  uint32_t bits;
+  memcpy(&bits, &f, sizeof bits);
+  return (uint16_t)(bits >> 16);
+}
+
 /* One output row: sequence b, node u, query head h.  Key set is the prefix in
  * column order followed by the walked ancestor rows in ascending row order. */
 static void attend_one(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                        int32_t ks, int32_t kl, const int32_t* par, int b, int u, int h, int M,
-                       int Hq, int Hkv, int D, double scale, double* o) {
+                       int Hq, int Hkv, int D, double scale, double rope_base, double* o) {
   const int G = Hq / Hkv, hk = h / G, n = M + 1;
   const uint16_t* qr = q + (((int64_t)b * n + u) * Hq + h) * D;
   const uint16_t* kb = k + ((int64_t)b * Hkv + hk) * S_cap * D;
   const uint16_t* vb = v + ((int64_t)b * Hkv + hk) * S_cap * D;
+  /* the query row, rotated to its position when a rotary base is given (the
+   * keys are used as stored: tree rows are rotated when they are written) */
+  double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int d = 0; d < D; ++d) qd[d] = bf16_to_double(qr[d]);
+  if (rope_base > 0.0) {
+    int depth_u = 0;
+    for (int x = u; x != 0; x = par[x]) ++depth_u;
+    rope_rotate(qd, D, (double)kl + depth_u, rope_base);
+  }
 
   /* explicit key list: prefix columns, then ancestor tree rows ascending */
   char* is_anc = (char*)calloc((size_t)n, 1);
@@ -148,7 +201,7 @@ static void attend_one(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
   for (t = 0; t < nkeys; ++t) {
     const uint16_t* kr = kb + cols[t] * D;
     double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += bf16_to_double(qr[d]) * bf16_to_double(kr[d]);
+    for (int d = 0; d < D; ++d) acc += qd[d] * bf16_to_double(kr[d]);
     s[t] = acc * scale;
     if (s[t] > mx) mx = s[t];
   }
@@ -161,29 +214,44 @@ static void attend_one(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     for (int d = 0; d < D; ++d) o[d] += p * bf16_to_double(vr[d]);
   }
   for (int d = 0; d < D; ++d) o[d] /= l;
+  free(qd);
   free(s);
   free(cols);
   free(is_anc);
 }
 
+/* One row of sequence b, or zeros if the sequence is invalid (status != 0 or
+ * a bad cache geometry). */
+static void attend_row_or_zero(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                               const int32_t* kv_start, const int32_t* kv_len, const int32_t* parent,
+                               const int32_t* status, int b, int u, int h, int M, int Hq, int Hkv, int D,
+                               double scale, double rope_base, double* o) {
+  if (status[b] != 0 || !geometry_ok(kv_start[b], kv_len[b], M, S_cap)) {
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    return;
+  }
+  attend_one(q, k, v, S_cap, kv_start[b], kv_len[b], parent + (int64_t)b * (M + 1), b, u, h, M, Hq, Hkv, D,
+             scale, rope_base, o);
+}
+
 /* Selected rows: sel is [nsel][3] = (b, u, h); out is [nsel][D].  Rows of an
- * invalid sequence (status != 0 or bad cache geometry) are zero. */
+ * invalid sequence (status != 0 or bad cache geometry) are zero.  rope_base > 0
+ * rotates each query row to position kv_len + depth(u) first (0: q is used as
+ * given).  (Rows are independent; the OpenMP pragmas only take effect in the
+ * benchmark's all-cores build.) */
 int oracle_tree_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                                const int32_t* kv_start, const int32_t* kv_len, const int32_t* parent,
                                const int32_t* status, int B, int M, int Hq, int Hkv, int D,
-                               double scale, const int32_t* sel, int64_t nsel, double* out) {
+                               double scale, double rope_base, const int32_t* sel, int64_t nsel, double* out) {
   if (Hkv <= 0 || Hq % Hkv != 0) return -1;
   for (int64_t i = 0; i < nsel; ++i) {
     int b = sel[3 * i], u = sel[3 * i + 1], h = sel[3 * i + 2];
-    double* o = out + i * D;
     if (b < 0 || b >= B || u < 0 || u > M || h < 0 || h >= Hq) return -2;
-    if (status[b] != 0 || !geometry_ok(kv_start[b], kv_len[b], M, S_cap)) {
-      for (int d = 0; d < D; ++d) o[d] = 0.0;
-      continue;
-    }
-    attend_one(q, k, v, S_cap, kv_start[b], kv_len[b], parent + (int64_t)b * (M + 1), b, u, h, M,
-               Hq, Hkv, D, scale, o);
   }
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nsel; ++i)
+    attend_row_or_zero(q, k, v, S_cap, kv_start, kv_len, parent, status, sel[3 * i], sel[3 * i + 1],
+                       sel[3 * i + 2], M, Hq, Hkv, D, scale, rope_base, out + i * D);
   return 0;
 }
 
@@ -191,17 +259,15 @@ int oracle_tree_attention_rows(const uint16_t* q, const uint16_t* k, const uint1
 int oracle_tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                           const int32_t* kv_start, const int32_t* kv_len, const int32_t* parent,
                           const int32_t* status, int B, int M, int Hq, int Hkv, int D, double scale,
-                          double* out) {
+                          double rope_base, double* out) {
   if (Hkv <= 0 || Hq % Hkv != 0) return -1;
-  for (int b = 0; b < B; ++b)
-    for (int u = 0; u <= M; ++u)
-      for (int h = 0; h < Hq; ++h) {
-        int32_t sel[3] = {b, u, h};
-        double* o = out + (((int64_t)b * (M + 1) + u) * Hq + h) * D;
-        int rc = oracle_tree_attention_rows(q, k, v, S_cap, kv_start, kv_len, parent, status, B, M,
-                                            Hq, Hkv, D, scale, sel, 1, o);
-        if (rc) return rc;
-      }
+  const int64_t rows = (int64_t)B * (M + 1) * Hq;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < rows; ++i) {
+    const int h = (int)(i % Hq), u = (int)((i / Hq) % (M + 1)), b = (int)(i / ((int64_t)Hq * (M + 1)));
+    attend_row_or_zero(q, k, v, S_cap, kv_start, kv_len, parent, status, b, u, h, M, Hq, Hkv, D, scale,
+                       rope_base, out + i * D);
+  }
   return 0;
 }
 
@@ -216,6 +282,7 @@ int oracle_tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* 
 
 /* First maximum wins (strict '>'). */
 int oracle_argmax_rows(const float* logits, int64_t rows, int V, int32_t* out) {
+#pragma omp parallel for
   for (int64_t r = 0; r < rows; ++r) {
     const float* x = logits + r * V;
     int best = 0;
@@ -400,10 +467,16 @@ int oracle_kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layer
  * layer.  tree_k / tree_v are [L][B][Hkv][M+1][D]; a sequence whose rows would
  * not fit the cache (or whose geometry is negative) is left untouched.
  * ------------------------------------------------------------------------- */
+/* depth [B][M+1] and rope_base > 0: each K row r is rotated to position
+ * kv_len + depth[b][r] (the rotary embedding above) and stored as the nearest
+ * bf16; V rows are copied as they are.  depth NULL or rope_base <= 0: plain copy. */
 int oracle_tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, const uint16_t* tree_k,
                          const uint16_t* tree_v, int L, int B, int Hkv, int D, int64_t S_cap, int M,
-                         const int32_t* kv_start, const int32_t* kv_len) {
+                         const int32_t* kv_start, const int32_t* kv_len, const int32_t* depth,
+                         double rope_base) {
   const int n = M + 1;
+  const int rope = depth != NULL && rope_base > 0.0;
+  double* row = (double*)malloc(sizeof(double) * (size_t)D);
   for (int l = 0; l < L; ++l)
     for (int b = 0; b < B; ++b) {
       if (!geometry_ok(kv_start[b], kv_len[b], M, S_cap)) continue;
@@ -412,11 +485,22 @@ int oracle_tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, c
           const int64_t src = ((((int64_t)l * B + b) * Hkv + h) * n + r) * D;
           const int64_t col = (int64_t)kv_start[b] + kv_len[b] + r;
           const int64_t dst = (((int64_t)b * Hkv + h) * S_cap + col) * D;
-          for (int d = 0; d < D; ++d) {
-            k_layers[l][dst + d] = tree_k[src + d];
-            v_layers[l][dst + d] = tree_v[src + d];
+          if (rope) {
+            for (int d = 0; d < D; ++d) row[d] = bf16_to_double(tree_k[src + d]);
+            rope_rotate(row, D, (double)kv_len[b] + depth[(int64_t)b * n + r], rope_base);
+            for (int d = 0; d < D; ++d) k_layers[l][dst + d] = double_to_bf16(row[d]);
+          } else {
+            for (int d = 0; d < D; ++d) k_layers[l][dst + d] = tree_k[src + d];
           }
+          for (int d = 0; d < D; ++d) v_layers[l][dst + d] = tree_v[src + d];
         }
     }
+  free(row);
+  return 0;
+}
+
+/* Nearest bf16 of each double (exported for its pins). */
+int oracle_round_bf16(const double* x, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = double_to_bf16(x[i]);
   return 0;
 }
