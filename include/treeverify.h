@@ -109,16 +109,34 @@ tv_status tree_build_mask(const int32_t* parent, int B, int M, int max_depth, ui
  *             the partial results of the key splits of one call; its contents
  *             need no initialisation and are dead after the call.  Calls that
  *             overlap on the device must not share a workspace.
+ *   flags     0 or TV_ATTN_PREFIX_READY (below); any other bit is an argument
+ *             error
  *   D in {64, 128}; Hq % Hkv == 0 (q head h reads kv head h / (Hq/Hkv));
  *   scale > 0 (normally 1/sqrt(D)).
  * Contract: the K/V rows inside each sequence's key range hold finite values.
  */
 size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64_t S_cap);
 
+/*
+ * TV_ATTN_PREFIX_READY -- the caller promises that the kernel launched just
+ * before this call on the same stream writes neither kv_start / kv_len nor any
+ * K/V column of the committed prefixes (it may write q, the tree rows, the
+ * ancestor masks or the status).  That holds for the attention call of the next
+ * layer, and after tree_kv_write or tree_build_mask.  The kernel may then read
+ * the geometry and start streaming prefix K/V tiles while that launch is still
+ * running; the tree rows, q, the masks and the status are read only after it
+ * has finished.  If the geometry turns out to have changed anyway, the affected
+ * sequences get zero rows and TV_SEQ_BAD_GEOMETRY instead of a wrong result.
+ * Never set it right after kv_commit_realign, which rewrites both.  The head
+ * dim 64 kernel ignores the flag.
+ */
+#define TV_ATTN_PREFIX_READY 1u
+
 tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                          const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                          int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
-                         uint16_t* out, void* workspace, size_t workspace_bytes, tv_stream_t stream);
+                         uint16_t* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                         tv_stream_t stream);
 
 /*
  * tree_attention_noalloc -- tree_attention for callers that cannot allocate
@@ -131,13 +149,17 @@ tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v
  * tree_attention_noalloc_max_scratch() bytes (32 MiB) compiled into the
  * library, which every GPU that loads the library holds until the process
  * exits.  A shape whose tree_attention_workspace_size exceeds that maximum is
- * rejected with TV_ERR_UNSUPPORTED; on a 148-SM GPU none does (the key split
- * stops once the query tiles fill the SMs, so the partials stay below about
- * 3 x 148 x 66,560 bytes).  Nothing is allocated: the first call on a
- * device only looks up the array's device address (make that first call before
- * any stream capture).  All calls share the one array, so calls that overlap on
- * the device race with each other; each call overwrites what it reads, so no
- * clearing is needed between calls.
+ * rejected with TV_ERR_UNSUPPORTED; on a 148-SM GPU none does (splits are
+ * added only while query tiles x splits stays within 2 CTAs per SM, so the
+ * partials stay within 2 x SMs x 128 rows x 130 floats = 19.7 MB on 148 SMs).
+ * Nothing is allocated: the first call on a device only looks up the array's
+ * device address and caches it (make that first call before any stream
+ * capture).  The cache assumes one primary context per device for the life of
+ * the process: after a cudaDeviceReset the address is stale, so do not call
+ * this entry point on a device that was reset.  All calls share the one array,
+ * so calls that overlap on the device race with each other; each call
+ * overwrites what it reads, so no clearing is needed between calls.  The
+ * launch flags of tree_attention are not offered here (flags = 0).
  */
 size_t tree_attention_noalloc_max_scratch(void);
 
@@ -231,6 +253,20 @@ int tv_last_cuda_error(void);
 
 /* ABI version (major * 100 + minor). */
 int tv_version(void);
+
+/*
+ * tv_set_wait_limit_ns -- testing hook for the timeout path of tree_attention
+ * (the pages have no counterpart).  Every device wait of the tensor-core
+ * attention kernel is bounded; this sets, for the launches that follow in this
+ * process, the limit of the pipeline waits (a stage that waits for the previous
+ * one: scores, probabilities, output, K/V tiles).  A wait that runs out makes
+ * the kernel give up on that sequence: its rows are zero and TV_SEQ_TIMEOUT is
+ * OR-ed into its status.  The waits that drain copies and MMAs still in flight
+ * before a CTA exits keep the full 1 s limit, so a short limit never leaves work
+ * behind.  ns = 0 restores the default (1 s); larger values are clamped to it.
+ * Not thread-safe with respect to launches on other threads.
+ */
+void tv_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -32,13 +32,13 @@ def host_u32(t):
     return t.cpu().numpy().view(np.uint32)
 
 
-def gpu_attention(q, k, v, kv_start, kv_len, anc, status, scale=None):
+def gpu_attention(q, k, v, kv_start, kv_len, anc, status, scale=None, flags=0):
     out = torch.full_like(q, float("nan"))
     B, n, Hq, D = q.shape
     ws = tv.attention_workspace(B, n - 1, Hq, k.shape[1], D, k.shape[2], q.device)
     if ws is not None:
         ws.fill_(0xFF)  # NaN patterns: the kernel must not depend on the workspace contents
-    tv.tree_attention(q, k, v, i32(kv_start), i32(kv_len), anc, status, out, ws, scale=scale)
+    tv.tree_attention(q, k, v, i32(kv_start), i32(kv_len), anc, status, out, ws, scale=scale, flags=flags)
     return out
 
 

@@ -26,9 +26,27 @@ def load_golden(name):
     return out
 
 
+# Raw error statistics of every attention comparison of the session, by label:
+# max |gpu - ref| over all elements, and max |gpu - ref| / |ref| over the
+# elements with |ref| >= 0.1 (the benchmark spec's max-abs / max-rel figures, which
+# the allclose bar above combines).  Printed at the end of the session.
+ERR_STATS = {}
+
+
+def error_stats(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= 0.1
+    return {"max_abs": float(err.max()) if err.size else 0.0,
+            "max_rel_ref_ge_0.1": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+            "elements": int(err.size)}
+
+
 def assert_attn_close(got, ref, what=""):
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
+    ERR_STATS[what or "attention"] = error_stats(got, ref)
     err = np.abs(got - ref)
     bad = err > ATOL + RTOL * np.abs(ref)
     if bad.any():

@@ -60,13 +60,16 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.tree_build_mask(z, 0, 4, 3, z, z, z, z) == 0
     # attention: Hq not a multiple of Hkv, unsupported head dim, bad scale, misaligned q
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 6, 4, 128,
-                              ctypes.c_float(0.1), dummy, z, 0, z) == 1
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 1
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 96,
-                              ctypes.c_float(0.1), dummy, z, 0, z) == 2
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 2
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
-                              ctypes.c_float(0.0), dummy, z, 0, z) == 1
+                              ctypes.c_float(0.0), dummy, z, 0, 0, z) == 1
     assert lib.tree_attention(P(258), dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
-                              ctypes.c_float(0.1), dummy, z, 0, z) == 1
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 1
+    # an unknown launch flag
+    assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
+                              ctypes.c_float(0.1), dummy, z, 0, 2, z) == 1
     # the workspace size is a pure function of the shape; D = 64 needs none
     assert lib.tree_attention_workspace_size(1, 64, 32, 32, 64, 2120) == 0
     assert lib.tree_attention_workspace_size(-1, 64, 32, 32, 128, 2120) == 0

@@ -19,12 +19,12 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _run(orc, q, k, v, parent, kv_start, kv_len, max_depth=1000, status_override=None, sel=None):
+def _run(orc, q, k, v, parent, kv_start, kv_len, max_depth=1000, status_override=None, sel=None, flags=0):
     par, anc, depth, status = gpu_mask(parent, max_depth)
     if status_override is not None:
         status.copy_(i32(status_override))
     st_h = status.cpu().numpy()
-    out = gpu_attention(q, k, v, kv_start, kv_len, anc, status)
+    out = gpu_attention(q, k, v, kv_start, kv_len, anc, status, flags=flags)
     torch.cuda.synchronize()
     qb, kb, vb = W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v)
     Hkv = k.shape[1]
@@ -74,7 +74,7 @@ def test_parity_full(orc, B, M, Hq, Hkv, D, P):
     q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, D, P, seed=B * 1000 + M)
     got, ref, _ = _run(orc, q, k, v, par, ks, kl)
     assert not np.isnan(got).any()
-    assert_attn_close(got, ref, "attention")
+    assert_attn_close(got, ref, f"B{B} M{M} Hq{Hq} Hkv{Hkv} D{D} P{P}")
 
 
 def test_left_padded_ragged(orc):
@@ -150,16 +150,24 @@ def test_invalid_sequences_zero_rows(orc):
     assert_attn_close(got, ref, "attention with invalid sequences")
 
 
+PREFIX_READY = 1
+
+
+@pytest.mark.parametrize("flags", [0, PREFIX_READY], ids=["plain", "prefix_ready"])
 @pytest.mark.parametrize("name", ["tiny", "mha7b", "eqspec"])
-def test_config_full(orc, name):
+def test_config_full(orc, name, flags):
+    """Every output row; with TV_ATTN_PREFIX_READY (tree_build_mask is the launch
+    just before) the prefix tiles are requested before the grid dependency, and
+    the result must not change."""
     cfg = W.CONFIGS[name]
     st = W.make_step(cfg, seed=0, device=dev(), with_logits=False)
-    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth)
-    assert_attn_close(got, ref, name)
+    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth, flags=flags)
+    assert_attn_close(got, ref, f"{name} ({'prefix_ready' if flags else 'plain'})")
 
 
+@pytest.mark.parametrize("flags", [0, PREFIX_READY], ids=["plain", "prefix_ready"])
 @pytest.mark.parametrize("name", ["b32gqa", "stress"])
-def test_config_sampled(orc, name):
+def test_config_sampled(orc, name, flags):
     cfg = W.CONFIGS[name]
     st = W.make_step(cfg, seed=0, device=dev(), with_logits=False)
     rng = np.random.default_rng(1)
@@ -167,5 +175,20 @@ def test_config_sampled(orc, name):
     sel = [(0, u, h) for u in range(n) for h in range(0, cfg.Hq, max(1, cfg.Hq // 8))]
     sel += [(int(rng.integers(cfg.B)), int(rng.integers(n)), int(rng.integers(cfg.Hq))) for _ in range(96)]
     sel = np.array(sel, np.int32)
-    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth, sel=sel)
-    assert_attn_close(got, ref, name)
+    got, ref, _ = _run(orc, st.q, st.k, st.v, st.parent, st.kv_start, st.kv_len, cfg.max_depth, sel=sel,
+                       flags=flags)
+    assert_attn_close(got, ref, f"{name} sampled ({'prefix_ready' if flags else 'plain'})")
+
+
+def test_prefix_ready_is_bit_identical(orc):
+    """The launch flag changes when the prefix tiles are requested, not what is
+    computed: outputs with and without it are equal bit for bit (eqspec shapes,
+    left-padded ragged prefixes; a ring's worth of tiles is requested early)."""
+    cfg = W.CONFIGS["eqspec"]
+    st = W.make_step(cfg, seed=5, device=dev(), with_logits=False)
+    par, anc, depth, status = gpu_mask(st.parent, cfg.max_depth)
+    a = gpu_attention(st.q, st.k, st.v, st.kv_start, st.kv_len, anc, status, flags=0)
+    b = gpu_attention(st.q, st.k, st.v, st.kv_start, st.kv_len, anc, status, flags=PREFIX_READY)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert int(status.abs().sum()) == 0

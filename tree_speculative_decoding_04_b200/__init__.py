@@ -7,6 +7,7 @@ tensors into those calls (``_lib``) and offers a host-side driver of one whole
 verification step (``verifier``).
 """
 from ._lib import (  # noqa: F401
+    ATTN_PREFIX_READY,
     EXPORTS,
     LIB_PATH,
     MAX_TREE_ROWS,
@@ -19,6 +20,7 @@ from ._lib import (  # noqa: F401
     kv_commit_realign,
     layer_pointers,
     load,
+    set_wait_limit_ns,
     tree_accept,
     tree_attention,
     tree_attention_workspace_size,

@@ -21,6 +21,7 @@ SEQ_TOO_DEEP = 2
 SEQ_TIMEOUT = 4
 SEQ_BAD_GEOMETRY = 8
 MAX_TREE_ROWS = 256
+ATTN_PREFIX_READY = 1
 
 EXPORTS = (
     "tree_build_mask",
@@ -34,6 +35,7 @@ EXPORTS = (
     "tv_status_string",
     "tv_last_cuda_error",
     "tv_version",
+    "tv_set_wait_limit_ns",
 )
 
 
@@ -56,7 +58,8 @@ def load(path: str = LIB_PATH):
     lib.tree_build_mask.argtypes = [P, i32, i32, i32, P, P, P, P]
     lib.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
     lib.tree_attention_workspace_size.restype = ctypes.c_size_t
-    lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, ctypes.c_size_t, P]
+    lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, ctypes.c_size_t,
+                                   ctypes.c_uint, P]
     lib.tree_attention_noalloc_max_scratch.argtypes = []
     lib.tree_attention_noalloc_max_scratch.restype = ctypes.c_size_t
     lib.tree_attention_noalloc.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
@@ -70,6 +73,8 @@ def load(path: str = LIB_PATH):
     lib.tv_status_string.restype = ctypes.c_char_p
     lib.tv_last_cuda_error.restype = ctypes.c_int
     lib.tv_version.restype = ctypes.c_int
+    lib.tv_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.tv_set_wait_limit_ns.restype = None
     _lib = lib
     return lib
 
@@ -132,9 +137,12 @@ def attention_workspace(B, M, Hq, Hkv, D, S_cap, device) -> torch.Tensor | None:
     return torch.empty((nbytes + 15) // 16 * 16, dtype=torch.uint8, device=device)
 
 
-def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=None, scale=None, stream=None):
+def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=None, scale=None, stream=None,
+                   flags=0):
     """q [B][M+1][Hq][D] bf16; k, v [B][Hkv][S_cap][D] bf16 (one layer) -> out like q.
-    workspace: a uint8 device tensor of at least tree_attention_workspace_size bytes."""
+    workspace: a uint8 device tensor of at least tree_attention_workspace_size bytes.
+    flags: 0 or ATTN_PREFIX_READY (the launch just before this one on the stream
+    writes neither the geometry nor any prefix K/V column)."""
     B, n, Hq, D = q.shape
     Hkv, S_cap = k.shape[1], k.shape[2]
     _need(q, torch.bfloat16, (B, n, Hq, D), "q")
@@ -150,7 +158,7 @@ def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=N
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load().tree_attention(_ptr(q), _ptr(k), _ptr(v), S_cap, _ptr(kv_start), _ptr(kv_len), _ptr(anc_mask),
                                _ptr(status), B, n - 1, Hq, Hkv, D, float(scale), _ptr(out), _ptr(workspace),
-                               ws_bytes, _stream(stream))
+                               ws_bytes, int(flags), _stream(stream))
     _check(rc, "tree_attention")
 
 
@@ -206,6 +214,12 @@ def tree_kv_write(k_layer_ptrs, v_layer_ptrs, tree_k, tree_v, S_cap, kv_start, k
     rc = load().tree_kv_write(_ptr(k_layer_ptrs), _ptr(v_layer_ptrs), _ptr(tree_k), _ptr(tree_v), L, B, Hkv, D,
                               int(S_cap), n - 1, _ptr(kv_start), _ptr(kv_len), _stream(stream))
     _check(rc, "tree_kv_write")
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Testing hook: limit (ns) of tree_attention's pipeline waits for later
+    launches; 0 restores the default (1 s)."""
+    load().tv_set_wait_limit_ns(int(ns))
 
 
 def layer_pointers(layers, device=None) -> torch.Tensor:

@@ -145,12 +145,12 @@ __global__ void __launch_bounds__(kMaxRows) accept_walk_kernel(
   const int64_t rbase = (int64_t)b * n;
   int32_t* pth = path + (int64_t)b * (max_depth + 1);
 
-  // Inputs not produced by the argmax kernel may be read before waiting on it:
-  // the argmax kernel triggers this launch only after its own wait returned,
-  // so everything launched before it has completed.
+  // parent, depth and draft are written by no kernel of the step after
+  // tree_build_mask, and the argmax kernel triggers this launch only after its
+  // own wait returned, so they may be read before waiting on it.  status may
+  // still gain a bit from the attention launches, so it is read after the wait.
   pdl_launch_dependents();
   const bool in = u < n;
-  const int st0 = status[b];
   const int p = in ? parent[rbase + u] : 0;
   const int dp = in ? depth[rbase + u] : 0;
   const int dr = in ? draft[rbase + u] : 0;
@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kMaxRows) accept_walk_kernel(
   const bool bad_dep = in && (dp < 0 || dp > max_depth || dp > M || (u == 0 && dp != 0));
   const int flag = (__syncthreads_or(bad_par) ? kSeqBadParent : 0) | (__syncthreads_or(bad_dep) ? kSeqTooDeep : 0);
   pdl_wait_primary();
+  const int st0 = status[b];
   if (st0 != 0 || flag != 0) {
     for (int j = u; j <= max_depth; j += blockDim.x) pth[j] = 0;
     if (u == 0) {

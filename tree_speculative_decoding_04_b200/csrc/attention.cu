@@ -428,28 +428,25 @@ tv_status run(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, cuda
 }  // namespace
 }  // namespace tv
 
-extern "C" size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64_t S_cap) {
-  using namespace tv;
-  if (B <= 0 || M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S_cap < 0 || D != 128) return 0;
-  if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return 0;
-  TcPlan plan;
-  if (plan_attention_tc(B, M, Hq, Hkv, S_cap, plan) != TV_OK) return 0;
-  return plan.ws_bytes;
-}
+namespace tv {
 
-extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
-                                    const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
-                                    int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
-                                    uint16_t* out, void* workspace, size_t workspace_bytes, tv_stream_t stream) {
-  using namespace tv;
+tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                            const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
+                            int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale, uint16_t* out,
+                            unsigned flags, AttnCall& call) {
+  call.nothing_to_do = false;
   if (B < 0 || M < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || !(scale > 0.f)) return TV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return TV_ERR_INVALID_ARG;
+  if ((flags & ~(unsigned)TV_ATTN_PREFIX_READY) != 0) return TV_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
   if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
-  if (B == 0) return TV_OK;
+  if (B == 0) {
+    call.nothing_to_do = true;
+    return TV_OK;
+  }
   if (!q || !k || !v || !kv_start || !kv_len || !anc_mask || !status || !out) return TV_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TV_ERR_INVALID_ARG;
-  AttnParams p;
+  AttnParams& p = call.p;
   p.q = q;
   p.kv_start = kv_start;
   p.kv_len = kv_len;
@@ -466,21 +463,46 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
   p.rows_total = p.G * (M + 1);
   p.nsplit = p.tiles_per_split = p.stages = p.v_stages = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.flags = flags;
+  p.wait_limit_ns = pipeline_wait_limit_ns();
   p.ws = nullptr;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap tmk, tmv;
-  if (!encode_kv_map(&tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&tmv, v, B * Hkv, S_cap, D))
+  if (!encode_kv_map(&call.tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&call.tmv, v, B * Hkv, S_cap, D))
     return TV_ERR_INVALID_ARG;
-  if (D == 64) return run<64>(tmk, tmv, p, s);  // warp-MMA kernel, merge through DSMEM
-  // head dim 128: tcgen05 tensor-core kernel
+  if (D == 128) return plan_attention_tc(B, M, Hq, Hkv, S_cap, call.plan);
+  return TV_OK;
+}
+
+tv_status launch_attention(AttnCall& call, int D, cudaStream_t s) {
+  if (D == 64) return run<64>(call.tmk, call.tmv, call.p, s);  // warp-MMA kernel, merge through DSMEM
+  return run_attention_tc(call.tmk, call.tmv, call.p, call.plan, s);  // tcgen05 kernel
+}
+
+}  // namespace tv
+
+extern "C" size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64_t S_cap) {
+  using namespace tv;
+  if (B <= 0 || M < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S_cap < 0 || D != 128) return 0;
+  if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return 0;
   TcPlan plan;
-  tv_status r = plan_attention_tc(B, M, Hq, Hkv, S_cap, plan);
-  if (r != TV_OK) return r;
-  if (plan.ws_bytes > 0) {
-    if (!workspace || workspace_bytes < plan.ws_bytes || !aligned16(workspace)) return TV_ERR_INVALID_ARG;
-    p.ws = static_cast<float*>(workspace);
+  if (plan_attention_tc(B, M, Hq, Hkv, S_cap, plan) != TV_OK) return 0;
+  return plan.ws_bytes;
+}
+
+extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                                    const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
+                                    int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
+                                    uint16_t* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                                    tv_stream_t stream) {
+  using namespace tv;
+  AttnCall call;
+  tv_status r = prepare_attention(q, k, v, S_cap, kv_start, kv_len, anc_mask, status, B, M, Hq, Hkv, D, scale,
+                                  out, flags, call);
+  if (r != TV_OK || call.nothing_to_do) return r;
+  if (D == 128 && call.plan.ws_bytes > 0) {
+    if (!workspace || workspace_bytes < call.plan.ws_bytes || !aligned16(workspace)) return TV_ERR_INVALID_ARG;
+    call.p.ws = static_cast<float*>(workspace);
   }
-  return run_attention_tc(tmk, tmv, p, plan, s);
+  return launch_attention(call, D, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -504,7 +526,10 @@ void* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name only stands in for it, so the address is looked up once per
-// device, with that device current, and cached.
+// device, with that device current, and cached.  The cache assumes that each
+// device keeps one primary context for the life of the process: after a
+// cudaDeviceReset the cached address would be stale, so a process that resets
+// a device must not call tree_attention_noalloc on it again.
 tv_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -531,45 +556,16 @@ extern "C" tv_status tree_attention_noalloc(const uint16_t* q, const uint16_t* k
                                             const uint32_t* anc_mask, int32_t* status, int B, int M, int Hq,
                                             int Hkv, int D, float scale, uint16_t* out, tv_stream_t stream) {
   using namespace tv;
-  if (B < 0 || M < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || !(scale > 0.f)) return TV_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return TV_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
-  if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
-  if (B == 0) return TV_OK;
-  if (!q || !k || !v || !kv_start || !kv_len || !anc_mask || !status || !out) return TV_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TV_ERR_INVALID_ARG;
-  AttnParams p;
-  p.q = q;
-  p.kv_start = kv_start;
-  p.kv_len = kv_len;
-  p.anc = anc_mask;
-  p.status = status;
-  p.out = out;
-  p.S_cap = S_cap;
-  p.B = B;
-  p.M = M;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.W = (M + 1 + 31) / 32;
-  p.rows_total = p.G * (M + 1);
-  p.nsplit = p.tiles_per_split = p.stages = p.v_stages = 0;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.ws = nullptr;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap tmk, tmv;
-  if (!encode_kv_map(&tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&tmv, v, B * Hkv, S_cap, D))
-    return TV_ERR_INVALID_ARG;
-  if (D == 64) return run<64>(tmk, tmv, p, s);  // this path keeps its partials on chip
-  TcPlan plan;
-  tv_status r = plan_attention_tc(B, M, Hq, Hkv, S_cap, plan);
-  if (r != TV_OK) return r;
-  if (plan.ws_bytes > 0) {
-    if (plan.ws_bytes > kNoAllocScratchBytes) return TV_ERR_UNSUPPORTED;  // shape too large for the fixed scratch
+  AttnCall call;
+  tv_status r = prepare_attention(q, k, v, S_cap, kv_start, kv_len, anc_mask, status, B, M, Hq, Hkv, D, scale,
+                                  out, 0u, call);
+  if (r != TV_OK || call.nothing_to_do) return r;
+  if (D == 128 && call.plan.ws_bytes > 0) {  // D = 64 keeps its partials on chip
+    if (call.plan.ws_bytes > kNoAllocScratchBytes) return TV_ERR_UNSUPPORTED;  // too large for the fixed scratch
     void* scratch = nullptr;
     r = noalloc_scratch(&scratch);
     if (r != TV_OK) return r;
-    p.ws = static_cast<float*>(scratch);
+    call.p.ws = static_cast<float*>(scratch);
   }
-  return run_attention_tc(tmk, tmv, p, plan, s);
+  return launch_attention(call, D, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -26,6 +26,8 @@ struct AttnParams {
   int stages;           // key-tile ring depth (K ring of the tensor-core kernel)
   int v_stages;         // V ring depth of the tensor-core kernel
   float scale_log2;     // softmax scale * log2(e)
+  unsigned flags;       // TV_ATTN_* launch flags
+  uint64_t wait_limit_ns;  // limit of the pipeline waits (the drain waits keep kWaitLimitNs)
   float* ws;            // split partials: [units][nsplit][128 rows][128] O, then [units][nsplit][128][2] (m, l)
 };
 
@@ -69,5 +71,19 @@ struct TcPlan {
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& plan);
 tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnParams p, const TcPlan& plan,
                            cudaStream_t s);
+
+// Argument checks and launch parameters shared by every tree-attention entry
+// point.  Returns TV_OK with *nothing_to_do set for an empty batch.
+struct AttnCall {
+  AttnParams p;
+  CUtensorMap tmk, tmv;
+  TcPlan plan;  // filled for D = 128
+  bool nothing_to_do;
+};
+tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
+                            const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
+                            int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale, uint16_t* out,
+                            unsigned flags, AttnCall& call);
+tv_status launch_attention(AttnCall& call, int D, cudaStream_t s);
 
 }  // namespace tv

@@ -157,11 +157,11 @@ __device__ __forceinline__ uint64_t anc_window(const uint32_t (&aw)[kMaxRows / 3
 // O += P_j V_j for key tile j (one thread), then release the K/V stage and
 // publish the new O.  Returns false if P_j never arrived.
 __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t t_s0, uint32_t t_o, int j,
-                                         int v_stages) {
+                                         int v_stages, uint64_t lim) {
   const uint32_t idesc_o = idesc_bf16(128, 128, 1);
   const int sb = j & 1, s = j % v_stages;
-  if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1)) return false;
-  if (!mbar_wait(&sh->v_full[s], (j / v_stages) & 1)) return false;
+  if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1, lim)) return false;
+  if (!mbar_wait(&sh->v_full[s], (j / v_stages) & 1, lim)) return false;
   tc_fence_after();
   const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
 #pragma unroll
@@ -219,21 +219,71 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
+  auto issue_k = [&](int i, int32_t ks_, int k_lo_) {
+    const int s = i % k_stages;
+    uint8_t* dst = k_ring + s * kTileBytes;
+    mbar_arrive_expect_tx(&sh->k_full[s], kTileBytes);
+    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks_ + k_lo_ + i * kKeyTile, bh);
+    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks_ + k_lo_ + i * kKeyTile, bh);
+  };
+  auto issue_v = [&](int i, int32_t ks_, int k_lo_) {
+    const int s = i % v_stages;
+    uint8_t* dst = v_ring + s * kTileBytes;
+    mbar_arrive_expect_tx(&sh->v_full[s], kTileBytes);
+    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks_ + k_lo_ + i * kKeyTile, bh);
+    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks_ + k_lo_ + i * kKeyTile, bh);
+  };
+  // This sequence's key tiles are dealt evenly over the splits (ragged batches
+  // would otherwise leave short sequences in one split).
+  auto split_range = [&](int32_t kl_, int& k_lo_, int& nt_) {
+    const int seq_tiles = (kl_ + p.M + 1 + kKeyTile - 1) / kKeyTile;
+    const int tps = (seq_tiles + p.nsplit - 1) / p.nsplit;
+    k_lo_ = split * tps * kKeyTile;
+    nt_ = max(0, min(tps, seq_tiles - split * tps));
+  };
   // With programmatic launch this CTA can be resident while the previous kernel
-  // is still finishing.  Until the grid dependency resolves, warm L2 with the
-  // first key tiles of this split and with this CTA's query rows.  A prefetch
-  // binds no value: a write of the previous kernel to the same lines lands in
-  // L2, which every later read goes through, so a stale geometry read here only
-  // wastes the prefetch (issued only for a geometry that fits the cache, so the
-  // coordinates stay inside the tensor).
-  if (warp == 0 && lane == 0) {
+  // is still finishing.
+  //  - TV_ATTN_PREFIX_READY: the caller guarantees that the previous launch on
+  //    the stream writes neither the geometry nor any prefix column, so the
+  //    geometry is read now and the first ring's worth of tiles that lie wholly
+  //    inside the prefix is requested into shared memory before the grid
+  //    dependency resolves.  Tiles reaching the tree rows, the query rows, the
+  //    ancestor rows and the status are read only after it.
+  //  - otherwise: only warm L2 with the first key tile of this split and with
+  //    this CTA's query rows.  A prefetch binds no value: a write of the
+  //    previous kernel to the same lines lands in L2, which every later read
+  //    goes through, so a stale geometry read here only wastes the prefetch
+  //    (issued only for a geometry that fits the cache, so the coordinates stay
+  //    inside the tensor).
+  const bool prefix_ready = (p.flags & TV_ATTN_PREFIX_READY) != 0;
+  // limit of the pipeline waits; the waits that drain copies or MMAs in flight
+  // before the CTA exits always keep the full limit
+  const uint64_t lim = p.wait_limit_ns;
+  int32_t ks = 0, kl = 0;
+  int npre_k = 0, npre_v = 0;  // tiles requested before the grid dependency
+  if (prefix_ready) {
+    ks = __ldcg(p.kv_start + b);
+    kl = __ldcg(p.kv_len + b);
+    if (aligned_ok && geometry_ok(ks, kl, p.M, p.S_cap)) {
+      int k_lo_pre, nt_pre;
+      split_range(kl, k_lo_pre, nt_pre);
+      const int n_prefix = max(0, min(nt_pre, (kl - k_lo_pre) / kKeyTile));  // tiles wholly inside the prefix
+      npre_k = min(n_prefix, k_stages);
+      npre_v = min(n_prefix, v_stages);
+      if (warp == 0 && lane == 0)  // the thread that initialised the barriers
+        for (int i = 0; i < max(npre_k, npre_v); ++i) {
+          if (i < npre_k) issue_k(i, ks, k_lo_pre);
+          if (i < npre_v) issue_v(i, ks, k_lo_pre);
+        }
+    }
+  } else if (warp == 0 && lane == 0) {
     const int32_t ks_h = __ldcg(p.kv_start + b), kl_h = __ldcg(p.kv_len + b);
     if (geometry_ok(ks_h, kl_h, p.M, p.S_cap)) {
-      const int st = (kl_h + p.M + 1 + kKeyTile - 1) / kKeyTile;
-      const int tp = (st + p.nsplit - 1) / p.nsplit;
-      const int nt = min(kPrefetchTiles, max(0, min(tp, st - split * tp)));
+      int k_lo_h, nt_h;
+      split_range(kl_h, k_lo_h, nt_h);
+      const int nt = min(kPrefetchTiles, nt_h);
       for (int i = 0; i < nt; ++i) {
-        const int row = ks_h + (split * tp + i) * kKeyTile;
+        const int row = ks_h + k_lo_h + i * kKeyTile;
         tma_prefetch_3d(&tmk, 0, row, bh);
         tma_prefetch_3d(&tmk, 64, row, bh);
         tma_prefetch_3d(&tmv, 0, row, bh);
@@ -251,38 +301,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   }
   pdl_wait_primary();
   pdl_launch_dependents();
-  const int32_t ks = p.kv_start[b];
-  const int32_t kl = p.kv_len[b];
-  const bool valid = aligned_ok && p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  // The geometry is read again after the dependency: if the caller's promise
+  // did not hold (it changed), the sequence is flagged instead of computed.
+  const int32_t ks_now = p.kv_start[b], kl_now = p.kv_len[b];
+  const bool broken_promise = prefix_ready && (ks_now != ks || kl_now != kl);
+  ks = ks_now;
+  kl = kl_now;
+  const bool valid =
+      aligned_ok && !broken_promise && p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
   const int N = kl + p.M + 1;
-  // this sequence's key tiles are dealt evenly over the splits (ragged batches
-  // would otherwise leave short sequences in one split)
-  const int seq_tiles = (N + kKeyTile - 1) / kKeyTile;
-  const int tps = (seq_tiles + p.nsplit - 1) / p.nsplit;
-  const int t0 = split * tps;
-  const int ntiles = valid ? max(0, min(tps, seq_tiles - t0)) : 0;
-  const int k_lo = t0 * kKeyTile;
+  int k_lo = 0, nt_geo = 0;
+  split_range(kl, k_lo, nt_geo);
+  const int ntiles = valid ? nt_geo : 0;
 
-  // The first ring's worth of K/V tiles and the Q tile are requested before the
-  // TMEM allocation barrier, so their memory latency overlaps the set-up.
-  auto issue_k = [&](int i) {
-    const int s = i % k_stages;
-    uint8_t* dst = k_ring + s * kTileBytes;
-    mbar_arrive_expect_tx(&sh->k_full[s], kTileBytes);
-    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks + k_lo + i * kKeyTile, bh);
-    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks + k_lo + i * kKeyTile, bh);
-  };
-  auto issue_v = [&](int i) {
-    const int s = i % v_stages;
-    uint8_t* dst = v_ring + s * kTileBytes;
-    mbar_arrive_expect_tx(&sh->v_full[s], kTileBytes);
-    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks + k_lo + i * kKeyTile, bh);
-    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks + k_lo + i * kKeyTile, bh);
-  };
-  if (warp == 0 && lane == 0)  // the thread that initialised the barriers
+  // The rest of the first ring's worth of K/V tiles and the Q tile are
+  // requested before the TMEM allocation barrier, so their memory latency
+  // overlaps the set-up.
+  if (warp == 0 && lane == 0)
     for (int i = 0; i < min(ntiles, max(k_stages, v_stages)); ++i) {
-      if (i < k_stages) issue_k(i);
-      if (i < v_stages) issue_v(i);
+      if (i < k_stages && i >= npre_k) issue_k(i, ks, k_lo);
+      if (i < v_stages && i >= npre_v) issue_v(i, ks, k_lo);
     }
   const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
   const int gr = qtile * kRows + r;
@@ -321,33 +359,37 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       // K_i waits for S_{i-k_stages} to finish, V_i for PV_{i-v_stages}; both
       // complete in the order this loop issues, so it never blocks early
       bool to = false;
-      int k_issued = min(ntiles, k_stages), v_issued = min(ntiles, v_stages);
+      // the first ring's worth is already requested (or, for a sequence found
+      // invalid after the grid dependency, only the tiles requested before it)
+      int k_issued = ntiles > 0 ? min(ntiles, k_stages) : npre_k;
+      int v_issued = ntiles > 0 ? min(ntiles, v_stages) : npre_v;
       for (int i = 0; i < ntiles && !to; ++i) {
         if (i >= k_stages) {
-          if (!mbar_wait(&sh->k_empty[i % k_stages], ((i / k_stages) - 1) & 1)) {
+          if (!mbar_wait(&sh->k_empty[i % k_stages], ((i / k_stages) - 1) & 1, lim)) {
             to = true;
             break;
           }
-          issue_k(i);
+          issue_k(i, ks, k_lo);
           ++k_issued;
         }
         if (i >= v_stages) {
-          if (!mbar_wait(&sh->v_empty[i % v_stages], ((i / v_stages) - 1) & 1)) {
+          if (!mbar_wait(&sh->v_empty[i % v_stages], ((i / v_stages) - 1) & 1, lim)) {
             to = true;
             break;
           }
-          issue_v(i);
+          issue_v(i, ks, k_lo);
           ++v_issued;
         }
       }
-      if (to) {
-        atomicExch(&sh->timed_out, 1);
-        // copies still in flight must land before this CTA's shared memory is released
-        for (int i = max(0, k_issued - k_stages); i < k_issued; ++i)
-          mbar_wait(&sh->k_full[i % k_stages], (i / k_stages) & 1);
-        for (int i = max(0, v_issued - v_stages); i < v_issued; ++i)
-          mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1);
-      }
+      if (to) atomicExch(&sh->timed_out, 1);
+      // Every copy this thread issued must land before the CTA's shared memory
+      // is released, whether or not a consumer waited for it (a consumer that
+      // gave up, or a sequence found invalid, leaves copies unconsumed).  The
+      // last issued tile of each slot decides, so one wait per slot suffices.
+      for (int i = max(0, k_issued - k_stages); i < k_issued; ++i)
+        mbar_wait(&sh->k_full[i % k_stages], (i / k_stages) & 1);
+      for (int i = max(0, v_issued - v_stages); i < v_issued; ++i)
+        mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -357,7 +399,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
         const int s = i % k_stages, sb = i & 1;
-        if (!mbar_wait(&sh->k_full[s], (i / k_stages) & 1)) {
+        if (!mbar_wait(&sh->k_full[s], (i / k_stages) & 1, lim)) {
           to = true;
           break;
         }
@@ -371,15 +413,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         }
         tc_commit(&sh->k_empty[s]);
         tc_commit(&sh->s_full[sb]);
-        if (i >= 1 && !issue_pv(sh, v_ring, t_s0, t_o, i - 1, v_stages)) to = true;
+        if (i >= 1 && !issue_pv(sh, v_ring, t_s0, t_o, i - 1, v_stages, lim)) to = true;
       }
-      if (!to && !issue_pv(sh, v_ring, t_s0, t_o, ntiles - 1, v_stages)) to = true;
-      if (to) {
-        atomicExch(&sh->timed_out, 1);
-        // let every MMA issued so far retire before TMEM and shared memory are released
-        tc_commit(&sh->drain);
-        mbar_wait(&sh->drain, 0);
-      }
+      if (!to && !issue_pv(sh, v_ring, t_s0, t_o, ntiles - 1, v_stages, lim)) to = true;
+      if (to) atomicExch(&sh->timed_out, 1);
+      // Every MMA issued so far retires before TMEM and shared memory are
+      // released, also when a softmax warp gave up before reading the last O.
+      tc_commit(&sh->drain);
+      mbar_wait(&sh->drain, 0);
     }
   }
 
@@ -394,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       const int sb = i & 1;
       // every wait that gates a TMEM access is decided for the whole warp: the
       // tcgen05.ld / tcgen05.st that follow are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (i >> 1) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (i >> 1) & 1, lim))) {
         to = true;
         break;
       }
@@ -433,7 +474,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         const bool scale_o = grow && m != -INFINITY;
         if (__any_sync(0xffffffffu, scale_o)) {
           // O holds earlier tiles: rescale once PV_{i-1} has landed
-          if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, lim))) {
             to = true;
             break;
           }
@@ -480,8 +521,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       const int kend = N - key0;
       if (kend < kKeyTile) {
         uint8_t* vt = v_ring + (i % v_stages) * kTileBytes;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1)))
-          to = true;  // V_i must have landed
+        if (!__all_sync(0xffffffffu, mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1, lim))) {
+          to = true;  // V_i must have landed before its rows are overwritten
+          break;
+        }
         const int first = max(kend, 0);
         for (int idx = r; idx < (kKeyTile - first) * 16; idx += kRows) {
           const int row = first + idx / 16, c = idx % 16;
@@ -497,7 +540,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     if (to) atomicExch(&sh->timed_out, 1);
     have = __all_sync(0xffffffffu, ntiles > 0 && !to && warp_live);
     if (ntiles > 0 && !to) {
-      if (!mbar_wait(&sh->o_ready[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1)) {
+      if (!mbar_wait(&sh->o_ready[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, lim)) {
         atomicExch(&sh->timed_out, 1);
         have = false;
       }
@@ -641,9 +684,24 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && (sh->timed_out || !aligned_ok)) atomicOr(&p.status[b], kSeqTimeout);
+  if (threadIdx.x == 0 && broken_promise) atomicOr(&p.status[b], kSeqBadGeometry);
 }
 
 }  // namespace
+
+// Tuning of the launch plan (compile-time, so that a sweep can rebuild with -D):
+//   TV_TC_SPLIT_FACTOR  key splits are added while units * splits stays within
+//                       this many CTAs per SM
+//   TV_TC_ONE_PER_SM    1: a grid that fits one wave gets one CTA per SM with
+//                       deeper rings; 0: every CTA stays within half an SM's
+//                       shared memory, so the next launch's CTAs can become
+//                       resident beside it and start streaming early
+#ifndef TV_TC_SPLIT_FACTOR
+#define TV_TC_SPLIT_FACTOR 2
+#endif
+#ifndef TV_TC_ONE_PER_SM
+#define TV_TC_ONE_PER_SM 1
+#endif
 
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& lp) {
   int dev = 0, sms = 148;
@@ -656,7 +714,9 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
   // Split the key range only while the query tiles alone leave SMs idle: a
   // split adds a merge, and past one CTA per SM it adds a partial second wave.
-  int ns = units >= sms ? 1 : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, (2LL * sms) / units));
+  int ns = units >= sms ? 1
+                        : (int)std::min<int64_t>(kMaxSplit_tc,
+                                                 std::max<int64_t>(1, ((int64_t)TV_TC_SPLIT_FACTOR * sms) / units));
   ns = std::min(ns, key_tiles);
   lp.tiles_per_split = (key_tiles + ns - 1) / ns;
   lp.nsplit = (key_tiles + lp.tiles_per_split - 1) / lp.tiles_per_split;
@@ -664,7 +724,7 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
   // never waits on a CTA that is itself waiting), else one CTA per SM.
   const int64_t ctas = units * lp.nsplit;
-  const bool two_per_sm = ctas > sms;
+  const bool two_per_sm = !TV_TC_ONE_PER_SM || ctas > sms;
   // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
   // one CTA per SM: K ring 3, V ring up to 6
   lp.stages = two_per_sm ? 2 : std::min(3, std::max(2, lp.tiles_per_split));

@@ -64,13 +64,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded wait on the phase with the given parity; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait on the phase with the given parity; false if it gave up (after
+// limit_ns, or kWaitLimitPolls polls, whichever comes first).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < kWaitLimitPolls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
   return false;
 }
@@ -150,6 +151,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------- host side
 // Records the last CUDA error for tv_last_cuda_error(); returns TV_ERR_CUDA.
 tv_status record_cuda_error(cudaError_t e);
+
+// Limit (ns) of the pipeline waits of the next attention launches
+// (tv_set_wait_limit_ns); kWaitLimitNs unless a test shortened it.
+uint64_t pipeline_wait_limit_ns();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

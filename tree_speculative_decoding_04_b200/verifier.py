@@ -78,7 +78,10 @@ class StepResult:
 
 class TreeVerifier:
     def __init__(self, B, M, Hq, Hkv, D, V, L, S_cap, max_depth, realign=False, device="cuda",
-                 k_layers=None, v_layers=None, with_mask_outputs=None):
+                 k_layers=None, v_layers=None, with_mask_outputs=None, commit_layers=None):
+        """k_layers / v_layers: the L per-layer caches (default: allocated here).
+        commit_layers: the indices of the layers kv_commit_realign moves (default
+        all); a caller whose layer list repeats a buffer commits each buffer once."""
         self.B, self.M, self.Hq, self.Hkv, self.D, self.V, self.L = B, M, Hq, Hkv, D, V, L
         self.S_cap, self.max_depth, self.realign = S_cap, max_depth, bool(realign)
         self.n = M + 1
@@ -105,6 +108,9 @@ class TreeVerifier:
         self.v = v_layers if v_layers is not None else [torch.zeros((B, Hkv, S_cap, D), **bf) for _ in range(L)]
         self.k_ptrs = tv.layer_pointers(self.k, dev)
         self.v_ptrs = tv.layer_pointers(self.v, dev)
+        ids = list(range(L)) if commit_layers is None else list(commit_layers)
+        self.k_commit_ptrs = tv.layer_pointers([self.k[i] for i in ids], dev)
+        self.v_commit_ptrs = tv.layer_pointers([self.v[i] for i in ids], dev)
         self.workspace = tv.attention_workspace(B, M, Hq, Hkv, D, S_cap, dev)
         self.argmax = torch.zeros((B, self.n), **i32)
         # accept results side by side, so that they come back in one copy
@@ -129,9 +135,15 @@ class TreeVerifier:
     def build_mask(self, stream=None):
         tv.tree_build_mask(self.parent, self.max_depth, self.anc, self.depth, self.status, stream)
 
-    def attention(self, layer, stream=None):
+    def attention(self, layer, stream=None, prefix_ready=False):
+        """tree_attention of one layer.  prefix_ready: the kernel launched just
+        before on `stream` writes neither the geometry nor any prefix K/V column
+        (true after tree_build_mask, tree_kv_write and the attention of another
+        layer; false after kv_commit_realign), so prefix tiles may stream while
+        it finishes."""
         tv.tree_attention(self.q[layer], self.k[layer], self.v[layer], self.kv_start, self.kv_len, self.anc,
-                          self.status, self.out[layer], self.workspace, stream=stream)
+                          self.status, self.out[layer], self.workspace, stream=stream,
+                          flags=tv.ATTN_PREFIX_READY if prefix_ready else 0)
 
     def write_tree_rows(self, layer, stream=None):
         """tree_k / tree_v of one layer -> the cache, behind each sequence's prefix."""
@@ -144,7 +156,8 @@ class TreeVerifier:
                        self.argmax, self.accept_len, self.path, self.bonus, stream)
 
     def commit(self, stream=None):
-        tv.kv_commit_realign(self.k_ptrs, self.v_ptrs, self.B, self.Hkv, self.D, self.S_cap, self.M, self.path,
+        tv.kv_commit_realign(self.k_commit_ptrs, self.v_commit_ptrs, self.B, self.Hkv, self.D, self.S_cap, self.M,
+                             self.path,
                              self.accept_len, self.status, self.max_depth, self.kv_start, self.kv_len,
                              self.max_len, int(self.realign), self.attn_mask, self.pos_ids, stream)
 
@@ -153,7 +166,7 @@ class TreeVerifier:
         rows' K/V must already be in the cache."""
         self.build_mask(stream)
         for layer in range(self.L):
-            self.attention(layer, stream)
+            self.attention(layer, stream, prefix_ready=True)  # follows tree_build_mask or the previous layer
         self.accept(stream)
         self.commit(stream)
         return StepResult(self.accept_len, self.path, self.bonus)
@@ -224,7 +237,7 @@ class TreeVerifier:
             for layer in range(self.L):
                 s.wait_event(ev[1 + layer])
                 self.write_tree_rows(layer, s)
-                self.attention(layer, s)
+                self.attention(layer, s, prefix_ready=True)  # follows tree_kv_write
             s.wait_event(ev[1 + self.L])
             self.accept(s)
             self.commit(s)
