@@ -407,6 +407,20 @@ def per_call_times(ver, cfg, stream, reps, reset):
     g_reset = capture(reset, stream)
     reset_ms = event_time(g_reset.replay, reps, stream)
     com_ms = max(com_ms - reset_ms, 1e-6)
+    # the fused rotary embedding: attention with the query rotation, and the
+    # tree-row append with and without the K rotation (graphs of L launches)
+    ver.rope_theta = 10000.0
+    attn_rope_ms = None
+    if cfg.D == 128:  # the rotation is fused into the head dim 128 kernel only
+        g_r = capture(lambda: [ver.attention(layer, stream, prefix_ready=True) for layer in range(L)], stream)
+        attn_rope_ms = event_time(g_r.replay, reps, stream) / L
+        del g_r
+    g_w = capture(lambda: [ver.write_tree_rows(layer, stream) for layer in range(L)], stream)
+    kvw_rope_ms = event_time(g_w.replay, reps, stream) / L
+    ver.rope_theta = 0.0
+    g_w0 = capture(lambda: [ver.write_tree_rows(layer, stream) for layer in range(L)], stream)
+    kvw_ms = event_time(g_w0.replay, reps, stream) / L
+    del g_w, g_w0
     # one attention launch alone (eager, after a synchronisation), median of 10
     singles = []
     for r in range(10):
@@ -420,7 +434,8 @@ def per_call_times(ver, cfg, stream, reps, reset):
         a1.synchronize()
         singles.append(a0.elapsed_time(a1))
     return dict(attn_ms=attn_ms, mask_ms=mask_ms, acc_ms=acc_ms, com_ms=com_ms, reset_ms=reset_ms,
-                attn_single_ms=statistics.median(singles))
+                attn_single_ms=statistics.median(singles), attn_rope_ms=attn_rope_ms, kvw_rope_ms=kvw_rope_ms,
+                kvw_ms=kvw_ms)
 
 
 def measure_step(args, cfg, world, device, steps, warmup, with_clock=False, with_e2e=False):
@@ -509,6 +524,13 @@ def measure_step(args, cfg, world, device, steps, warmup, with_clock=False, with
                          "tree_attention_single_launch": t["attn_single_ms"] * 1e3,
                          "tree_accept": t["acc_ms"] * 1e3, "kv_commit_realign": t["com_ms"] * 1e3,
                          "geometry_reset_copies": t["reset_ms"] * 1e3},
+        "rope": {"attention_per_layer_us": t["attn_rope_ms"] * 1e3 if t["attn_rope_ms"] else None,
+                 "attention_plain_per_layer_us": t["attn_ms"] * 1e3,
+                 "attention_overhead_frac": t["attn_rope_ms"] / t["attn_ms"] - 1.0 if t["attn_rope_ms"] else None,
+                 "tree_kv_write_per_layer_us": t["kvw_rope_ms"] * 1e3,
+                 "tree_kv_write_plain_per_layer_us": t["kvw_ms"] * 1e3,
+                 "note": "query rows rotated to kv_len + depth while staged (TV_ATTN_ROPE); tree K rows rotated "
+                         "by tree_kv_write; base 10000"},
         "gpu_launches_per_step": ver.launches_per_step(),
         "_kv_len": [int(x) for x in kl_h],
     }

@@ -109,8 +109,13 @@ tv_status tree_build_mask(const int32_t* parent, int B, int M, int max_depth, ui
  *             the partial results of the key splits of one call; its contents
  *             need no initialisation and are dead after the call.  Calls that
  *             overlap on the device must not share a workspace.
- *   flags     0 or TV_ATTN_PREFIX_READY (below); any other bit is an argument
- *             error
+ *   flags     0 or an OR of TV_ATTN_PREFIX_READY and TV_ATTN_ROPE (below); any
+ *             other bit is an argument error
+ *   depth     int32 [B][M+1] node depths (from tree_build_mask); read only with
+ *             TV_ATTN_ROPE, may be NULL otherwise
+ *   rope_theta  rotary base (> 1, e.g. 10000), TV_ATTN_ROPE only
+ *   slot, n_slots  optional cache-slot map (see "Slot map" below); slot = NULL
+ *             means batch row b uses cache slot b (n_slots is then ignored)
  *   D in {64, 128}; Hq % Hkv == 0 (q head h reads kv head h / (Hq/Hkv));
  *   scale > 0 (normally 1/sqrt(D)).
  * Contract: the K/V rows inside each sequence's key range hold finite values.
@@ -121,8 +126,9 @@ size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64
  * TV_ATTN_PREFIX_READY -- the caller promises that the kernel launched just
  * before this call on the same stream writes neither kv_start / kv_len nor any
  * K/V column of the committed prefixes (it may write q, the tree rows, the
- * ancestor masks or the status).  That holds for the attention call of the next
- * layer, and after tree_kv_write or tree_build_mask.  The kernel may then read
+ * ancestor masks, the depths or the status; not the slot map).  That holds for
+ * the attention call of the next layer, and after tree_kv_write or
+ * tree_build_mask.  The kernel may then read
  * the geometry and start streaming prefix K/V tiles while that launch is still
  * running; the tree rows, q, the masks and the status are read only after it
  * has finished.  If the geometry turns out to have changed anyway, the affected
@@ -132,10 +138,37 @@ size_t tree_attention_workspace_size(int B, int M, int Hq, int Hkv, int D, int64
  */
 #define TV_ATTN_PREFIX_READY 1u
 
+/*
+ * TV_ATTN_ROPE -- q is given before its rotary position embedding: each query
+ * row of node u is rotated to position kv_len[b] + depth[b][u] while it is
+ * staged (the tree positions of "Batch Speculative Decoding Done Right",
+ * methodology: position-ID contiguity -- the prefix holds positions 0 ..
+ * kv_len-1 and every root-to-node path continues it without a gap).  Rotation:
+ * the pair (x[i], x[i + D/2]), i < D/2, turns by pos * rope_theta^(-2i/D)
+ * (half-split rotary embedding); the rotated row is rounded to bf16.  The keys
+ * are used as stored: write the tree rows with tree_kv_write's rotation.  Head
+ * dim 128 only (TV_ERR_UNSUPPORTED for 64).
+ */
+#define TV_ATTN_ROPE 2u
+
+/*
+ * Slot map (tree_attention, tree_kv_write, kv_commit_realign).  With slot !=
+ * NULL (int32 [B], device), the cache is a pool of n_slots sequences, each layer
+ * bf16 [n_slots][Hkv][S_cap][D], and batch row b uses slot slot[b]; kv_start,
+ * kv_len (and attn_mask / pos_ids rows) are indexed by slot, [n_slots], while
+ * the step's per-row arrays (q, out, parent, anc_mask, depth, status, path,
+ * accept_len, tree rows) stay indexed by batch row.  A batch can so be any set
+ * of the pool's sequences without moving their caches (the cross-batch
+ * scheduling of "Batch Speculative Decoding Done Right", methodology: EXSPEC
+ * groups sequences of equal length).  The slots of one batch must be distinct;
+ * a slot outside [0, n_slots) gets TV_SEQ_BAD_GEOMETRY and is skipped.
+ */
+
 tv_status tree_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                          const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                          int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
                          uint16_t* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                         const int32_t* depth, float rope_theta, const int32_t* slot, int n_slots,
                          tv_stream_t stream);
 
 /*
@@ -200,7 +233,8 @@ tv_status tree_accept(const float* logits, const int32_t* draft, const int32_t* 
  * For sequence b with n_b = accept_len[b] + 1 committed rows (0 if rejected):
  *   new content = old content ++ { tail row path[b][j] : j < n_b }, where the
  *   tail is the M+1 tree rows behind the content; kv_len[b] += n_b.
- *   realign = 0  per-sequence lengths: content stays at kv_start[b].
+ *   realign = 0  per-sequence lengths: content stays at kv_start[b] (with a
+ *                slot map, b's slot).
  *   realign = 1  left-padded: with Lmax' = max_b kv_len'[b], content moves to
  *                [Lmax' - kv_len'[b], Lmax'); kv_start'[b] = Lmax' - kv_len'[b].
  * All sources are read before they are overwritten (moves are in place).
@@ -215,12 +249,15 @@ tv_status tree_accept(const float* logits, const int32_t* draft, const int32_t* 
  *   attn_mask uint8 [B][S_cap], pos_ids int32 [B][S_cap]   out, may be NULL:
  *             mask = 1 on the new content columns, pos = column - kv_start',
  *             0 elsewhere
+ *   slot, n_slots  optional slot map (see tree_attention); with a map the
+ *             repad is over the batch's sequences only and Lmax' is theirs
  */
 tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers, int L, int B,
                             int Hkv, int D, int64_t S_cap, int M, const int32_t* path,
                             const int32_t* accept_len, int32_t* status, int max_depth,
                             int32_t* kv_start, int32_t* kv_len, int32_t* max_len, int realign,
-                            uint8_t* attn_mask, int32_t* pos_ids, tv_stream_t stream);
+                            uint8_t* attn_mask, int32_t* pos_ids, const int32_t* slot, int n_slots,
+                            tv_stream_t stream);
 
 /*
  * tree_kv_write -- place the K and V rows of the current step's M+1 tree nodes
@@ -236,6 +273,11 @@ tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers
  *   tree_k, tree_v  bf16 [L][B][Hkv][M+1][D] in (16-byte aligned)
  *   kv_start, kv_len  int32 [B] in: row r of sequence b goes to column
  *             kv_start[b] + kv_len[b] + r
+ *   depth     int32 [B][M+1] or NULL: with depths, each K row r is rotated to
+ *             position kv_len[b] + depth[b][r] (the rotation of TV_ATTN_ROPE,
+ *             base rope_theta > 1) and stored as bf16; V rows are copied as they
+ *             are.  NULL: K and V are copied as they are (rope_theta ignored).
+ *   slot, n_slots  optional slot map (see tree_attention)
  *   D in {64, 128}; 0 <= M < 256.
  * A sequence whose geometry breaks 0 <= kv_start, 0 <= kv_len,
  * kv_start + kv_len + M + 1 <= S_cap is left untouched (tree_attention then
@@ -243,7 +285,8 @@ tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* const* v_layers
  */
 tv_status tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, const uint16_t* tree_k,
                         const uint16_t* tree_v, int L, int B, int Hkv, int D, int64_t S_cap, int M,
-                        const int32_t* kv_start, const int32_t* kv_len, tv_stream_t stream);
+                        const int32_t* kv_start, const int32_t* kv_len, const int32_t* depth, float rope_theta,
+                        const int32_t* slot, int n_slots, tv_stream_t stream);
 
 /* Human-readable name of a tv_status. */
 const char* tv_status_string(tv_status s);

@@ -60,16 +60,24 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.tree_build_mask(z, 0, 4, 3, z, z, z, z) == 0
     # attention: Hq not a multiple of Hkv, unsupported head dim, bad scale, misaligned q
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 6, 4, 128,
-                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 1
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z, ctypes.c_float(0), z, 0, z) == 1
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 96,
-                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 2
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z, ctypes.c_float(0), z, 0, z) == 2
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
-                              ctypes.c_float(0.0), dummy, z, 0, 0, z) == 1
+                              ctypes.c_float(0.0), dummy, z, 0, 0, z, ctypes.c_float(0), z, 0, z) == 1
     assert lib.tree_attention(P(258), dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
-                              ctypes.c_float(0.1), dummy, z, 0, 0, z) == 1
-    # an unknown launch flag
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z, ctypes.c_float(0), z, 0, z) == 1
+    # an unknown launch flag; rotation without depths, without a base, or at head dim 64; a slot map of no slots
     assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
-                              ctypes.c_float(0.1), dummy, z, 0, 2, z) == 1
+                              ctypes.c_float(0.1), dummy, z, 0, 4, z, ctypes.c_float(0), z, 0, z) == 1
+    assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
+                              ctypes.c_float(0.1), dummy, z, 0, 2, z, ctypes.c_float(1e4), z, 0, z) == 1
+    assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
+                              ctypes.c_float(0.1), dummy, z, 0, 2, dummy, ctypes.c_float(0.5), z, 0, z) == 1
+    assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 64,
+                              ctypes.c_float(0.1), dummy, z, 0, 2, dummy, ctypes.c_float(1e4), z, 0, z) == 2
+    assert lib.tree_attention(dummy, dummy, dummy, 64, dummy, dummy, dummy, dummy, 1, 3, 8, 4, 128,
+                              ctypes.c_float(0.1), dummy, z, 0, 0, z, ctypes.c_float(0), dummy, 0, z) == 1
     # the workspace size is a pure function of the shape; D = 64 needs none
     assert lib.tree_attention_workspace_size(1, 64, 32, 32, 64, 2120) == 0
     assert lib.tree_attention_workspace_size(-1, 64, 32, 32, 128, 2120) == 0
@@ -77,16 +85,27 @@ def test_argument_errors_are_synchronous(lib):
     assert lib.tree_accept(dummy, dummy, dummy, dummy, dummy, dummy, 1, 3, 0, 3, dummy, dummy, dummy, dummy, z) == 1
     # commit: bad realign flag, unsupported D
     assert lib.kv_commit_realign(dummy, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, dummy, 3, dummy, dummy, dummy, 2,
-                                 z, z, z) == 1
+                                 z, z, z, 0, z) == 1
     assert lib.kv_commit_realign(dummy, dummy, 1, 1, 1, 80, 64, 3, dummy, dummy, dummy, 3, dummy, dummy, dummy, 0,
-                                 z, z, z) == 2
+                                 z, z, z, 0, z) == 2
+    # commit: a slot map of no slots
+    assert lib.kv_commit_realign(dummy, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, dummy, 3, dummy, dummy, dummy, 0,
+                                 z, z, dummy, 0, z) == 1
     # tree-row append: negative size, unsupported D, tree too large, null rows, misaligned rows, empty
-    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, -1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
-    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 96, 64, 3, dummy, dummy, z) == 2
-    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 128, 512, 256, dummy, dummy, z) == 2
-    assert lib.tree_kv_write(dummy, dummy, z, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
-    assert lib.tree_kv_write(dummy, dummy, P(264), dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z) == 1
-    assert lib.tree_kv_write(z, z, z, z, 0, 1, 1, 128, 64, 3, z, z, z) == 0
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, -1, 1, 1, 128, 64, 3, dummy, dummy, z,
+                             ctypes.c_float(0), z, 0, z) == 1
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 96, 64, 3, dummy, dummy, z,
+                             ctypes.c_float(0), z, 0, z) == 2
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 128, 512, 256, dummy, dummy, z,
+                             ctypes.c_float(0), z, 0, z) == 2
+    assert lib.tree_kv_write(dummy, dummy, z, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z,
+                             ctypes.c_float(0), z, 0, z) == 1
+    assert lib.tree_kv_write(dummy, dummy, P(264), dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, z,
+                             ctypes.c_float(0), z, 0, z) == 1
+    assert lib.tree_kv_write(z, z, z, z, 0, 1, 1, 128, 64, 3, z, z, z, ctypes.c_float(0), z, 0, z) == 0
+    # tree-row append: rotation without a base
+    assert lib.tree_kv_write(dummy, dummy, dummy, dummy, 1, 1, 1, 128, 64, 3, dummy, dummy, dummy, ctypes.c_float(0),
+                             z, 0, z) == 1
 
 
 def test_binding_refuses_host_tensors():

@@ -8,6 +8,7 @@ verification step (``verifier``).
 """
 from ._lib import (  # noqa: F401
     ATTN_PREFIX_READY,
+    ATTN_ROPE,
     EXPORTS,
     LIB_PATH,
     MAX_TREE_ROWS,

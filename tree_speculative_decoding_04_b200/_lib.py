@@ -22,6 +22,7 @@ SEQ_TIMEOUT = 4
 SEQ_BAD_GEOMETRY = 8
 MAX_TREE_ROWS = 256
 ATTN_PREFIX_READY = 1
+ATTN_ROPE = 2
 
 EXPORTS = (
     "tree_build_mask",
@@ -59,14 +60,14 @@ def load(path: str = LIB_PATH):
     lib.tree_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
     lib.tree_attention_workspace_size.restype = ctypes.c_size_t
     lib.tree_attention.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P, ctypes.c_size_t,
-                                   ctypes.c_uint, P]
+                                   ctypes.c_uint, P, f32, P, i32, P]
     lib.tree_attention_noalloc_max_scratch.argtypes = []
     lib.tree_attention_noalloc_max_scratch.restype = ctypes.c_size_t
     lib.tree_attention_noalloc.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
     lib.tree_attention_noalloc.restype = ctypes.c_int
     lib.tree_accept.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, P]
-    lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P]
-    lib.tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P]
+    lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P, i32, P]
+    lib.tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P, f32, P, i32, P]
     for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign", "tree_kv_write"):
         getattr(lib, name).restype = ctypes.c_int
     lib.tv_status_string.argtypes = [ctypes.c_int]
@@ -138,18 +139,26 @@ def attention_workspace(B, M, Hq, Hkv, D, S_cap, device) -> torch.Tensor | None:
 
 
 def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=None, scale=None, stream=None,
-                   flags=0):
+                   flags=0, depth=None, rope_theta=0.0, slot=None):
     """q [B][M+1][Hq][D] bf16; k, v [B][Hkv][S_cap][D] bf16 (one layer) -> out like q.
     workspace: a uint8 device tensor of at least tree_attention_workspace_size bytes.
-    flags: 0 or ATTN_PREFIX_READY (the launch just before this one on the stream
-    writes neither the geometry nor any prefix K/V column)."""
+    flags: an OR of ATTN_PREFIX_READY (the launch just before this one on the
+    stream writes neither the geometry, the slot map nor any prefix K/V column)
+    and ATTN_ROPE (q is rotated to kv_len + depth[b][u] with base rope_theta).
+    slot: int32 [B] cache slots; k, v are then a pool [n_slots][Hkv][S_cap][D]
+    and kv_start / kv_len are [n_slots]."""
     B, n, Hq, D = q.shape
     Hkv, S_cap = k.shape[1], k.shape[2]
+    NS = k.shape[0] if slot is not None else B
     _need(q, torch.bfloat16, (B, n, Hq, D), "q")
-    _need(k, torch.bfloat16, (B, Hkv, S_cap, D), "k")
-    _need(v, torch.bfloat16, (B, Hkv, S_cap, D), "v")
-    _need(kv_start, torch.int32, (B,), "kv_start")
-    _need(kv_len, torch.int32, (B,), "kv_len")
+    _need(k, torch.bfloat16, (NS, Hkv, S_cap, D), "k")
+    _need(v, torch.bfloat16, (NS, Hkv, S_cap, D), "v")
+    _need(kv_start, torch.int32, (NS,), "kv_start")
+    _need(kv_len, torch.int32, (NS,), "kv_len")
+    if slot is not None:
+        _need(slot, torch.int32, (B,), "slot")
+    if flags & ATTN_ROPE:
+        _need(depth, torch.int32, (B, n), "depth")
     _need(anc_mask, torch.int32, (B, n, (n + 31) // 32), "anc_mask")
     _need(status, torch.int32, (B,), "status")
     _need(out, torch.bfloat16, (B, n, Hq, D), "out")
@@ -158,7 +167,8 @@ def tree_attention(q, k, v, kv_start, kv_len, anc_mask, status, out, workspace=N
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load().tree_attention(_ptr(q), _ptr(k), _ptr(v), S_cap, _ptr(kv_start), _ptr(kv_len), _ptr(anc_mask),
                                _ptr(status), B, n - 1, Hq, Hkv, D, float(scale), _ptr(out), _ptr(workspace),
-                               ws_bytes, int(flags), _stream(stream))
+                               ws_bytes, int(flags), _ptr(depth) if flags & ATTN_ROPE else None,
+                               float(rope_theta), _ptr(slot), NS, _stream(stream))
     _check(rc, "tree_attention")
 
 
@@ -180,39 +190,55 @@ def tree_accept(logits, draft, parent, depth, anc_mask, status, max_depth, argma
 
 
 def kv_commit_realign(k_layer_ptrs, v_layer_ptrs, B, Hkv, D, S_cap, M, path, accept_len, status, max_depth,
-                      kv_start, kv_len, max_len, realign, attn_mask=None, pos_ids=None, stream=None):
+                      kv_start, kv_len, max_len, realign, attn_mask=None, pos_ids=None, stream=None, slot=None):
     """k_layer_ptrs / v_layer_ptrs: int64 CUDA tensors [L] of layer base addresses
-    (each layer a bf16 [B][Hkv][S_cap][D] buffer)."""
+    (each layer a bf16 [B][Hkv][S_cap][D] buffer, or a pool [n_slots][Hkv][S_cap][D]
+    with slot: int32 [B] cache slots, kv_start / kv_len / mask rows per slot)."""
     L = k_layer_ptrs.numel()
+    NS = kv_start.shape[0] if slot is not None else B
     _need(k_layer_ptrs, torch.int64, (L,), "k_layer_ptrs")
     _need(v_layer_ptrs, torch.int64, (L,), "v_layer_ptrs")
     _need(path, torch.int32, (B, int(max_depth) + 1), "path")
-    for t, name in ((accept_len, "accept_len"), (status, "status"), (kv_start, "kv_start"), (kv_len, "kv_len")):
+    for t, name in ((accept_len, "accept_len"), (status, "status")):
         _need(t, torch.int32, (B,), name)
+    for t, name in ((kv_start, "kv_start"), (kv_len, "kv_len")):
+        _need(t, torch.int32, (NS,), name)
+    if slot is not None:
+        _need(slot, torch.int32, (B,), "slot")
     _need(max_len, torch.int32, (1,), "max_len")
     if attn_mask is not None:
-        _need(attn_mask, torch.uint8, (B, S_cap), "attn_mask")
+        _need(attn_mask, torch.uint8, (NS, S_cap), "attn_mask")
     if pos_ids is not None:
-        _need(pos_ids, torch.int32, (B, S_cap), "pos_ids")
+        _need(pos_ids, torch.int32, (NS, S_cap), "pos_ids")
     rc = load().kv_commit_realign(_ptr(k_layer_ptrs), _ptr(v_layer_ptrs), L, B, Hkv, D, int(S_cap), M, _ptr(path),
                                   _ptr(accept_len), _ptr(status), int(max_depth), _ptr(kv_start), _ptr(kv_len),
-                                  _ptr(max_len), int(realign), _ptr(attn_mask), _ptr(pos_ids), _stream(stream))
+                                  _ptr(max_len), int(realign), _ptr(attn_mask), _ptr(pos_ids), _ptr(slot), NS,
+                                  _stream(stream))
     _check(rc, "kv_commit_realign")
 
 
-def tree_kv_write(k_layer_ptrs, v_layer_ptrs, tree_k, tree_v, S_cap, kv_start, kv_len, stream=None):
+def tree_kv_write(k_layer_ptrs, v_layer_ptrs, tree_k, tree_v, S_cap, kv_start, kv_len, stream=None, depth=None,
+                  rope_theta=0.0, slot=None):
     """tree_k / tree_v bf16 [L][B][Hkv][M+1][D] -> the cache of every layer, at
     columns kv_start + kv_len + r (k_layer_ptrs / v_layer_ptrs as for
-    kv_commit_realign)."""
+    kv_commit_realign).  depth int32 [B][M+1]: K rows are rotated to kv_len +
+    depth with base rope_theta.  slot: int32 [B] cache slots of a pool (kv_start /
+    kv_len then [n_slots])."""
     L, B, Hkv, n, D = tree_k.shape
+    NS = kv_start.shape[0] if slot is not None else B
     _need(k_layer_ptrs, torch.int64, (L,), "k_layer_ptrs")
     _need(v_layer_ptrs, torch.int64, (L,), "v_layer_ptrs")
     _need(tree_k, torch.bfloat16, (L, B, Hkv, n, D), "tree_k")
     _need(tree_v, torch.bfloat16, (L, B, Hkv, n, D), "tree_v")
-    _need(kv_start, torch.int32, (B,), "kv_start")
-    _need(kv_len, torch.int32, (B,), "kv_len")
+    _need(kv_start, torch.int32, (NS,), "kv_start")
+    _need(kv_len, torch.int32, (NS,), "kv_len")
+    if depth is not None:
+        _need(depth, torch.int32, (B, n), "depth")
+    if slot is not None:
+        _need(slot, torch.int32, (B,), "slot")
     rc = load().tree_kv_write(_ptr(k_layer_ptrs), _ptr(v_layer_ptrs), _ptr(tree_k), _ptr(tree_v), L, B, Hkv, D,
-                              int(S_cap), n - 1, _ptr(kv_start), _ptr(kv_len), _stream(stream))
+                              int(S_cap), n - 1, _ptr(kv_start), _ptr(kv_len), _ptr(depth), float(rope_theta),
+                              _ptr(slot), NS, _stream(stream))
     _check(rc, "tree_kv_write")
 
 

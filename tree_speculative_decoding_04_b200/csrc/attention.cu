@@ -106,9 +106,11 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(co
   pdl_launch_dependents();
   __syncthreads();
 
-  const int32_t ks = p.kv_start[b];
-  const int32_t kl = p.kv_len[b];
-  const bool valid = p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int sl = cache_slot(p.slot, b, p.n_slots);  // cache slot of this batch row
+  const int32_t ks = sl >= 0 ? p.kv_start[sl] : 0;
+  const int32_t kl = sl >= 0 ? p.kv_len[sl] : 0;
+  const bool valid = sl >= 0 && p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int zc = sl * p.Hkv + hk;  // tensor-map row block of this (slot, kv head)
   const int N = kl + p.M + 1;  // keys of this sequence
   const int t0 = split * p.tiles_per_split;
   const int ntiles = valid ? max(0, min(p.tiles_per_split, (N + KT - 1) / KT - t0)) : 0;
@@ -130,8 +132,8 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(co
         uint8_t* kt = smem + (size_t)s * kStageBytes;
 #pragma unroll
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(kt + bx * kBoxBytes, &tmk, &full[s], bx * 64, col, bh);
-          tma_load_3d(kt + kTileBytes + bx * kBoxBytes, &tmv, &full[s], bx * 64, col, bh);
+          tma_load_3d(kt + bx * kBoxBytes, &tmk, &full[s], bx * 64, col, zc);
+          tma_load_3d(kt + kTileBytes + bx * kBoxBytes, &tmv, &full[s], bx * 64, col, zc);
         }
         ++issued;
       }
@@ -308,6 +310,7 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(co
     }
     __syncthreads();
     if (threadIdx.x == 0 && timed_out) atomicOr(&p.status[b], kSeqTimeout);
+    if (threadIdx.x == 0 && sl < 0) atomicOr(&p.status[b], kSeqBadGeometry);
     return;
   }
 
@@ -361,6 +364,7 @@ __global__ void __launch_bounds__((kMaxCWarps + 1) * 32) tree_attn_mma_kernel(co
   }
   cluster.sync();  // peers may still be reading this CTA's shared memory
   if (threadIdx.x == 0 && timed_out) atomicOr(&p.status[b], kSeqTimeout);
+  if (threadIdx.x == 0 && sl < 0) atomicOr(&p.status[b], kSeqBadGeometry);
 }
 
 struct LaunchPlan {
@@ -433,12 +437,17 @@ namespace tv {
 tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                             const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                             int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale, uint16_t* out,
-                            unsigned flags, AttnCall& call) {
+                            unsigned flags, const int32_t* depth, float rope_theta, const int32_t* slot,
+                            int n_slots, AttnCall& call) {
   call.nothing_to_do = false;
   if (B < 0 || M < 0 || Hq <= 0 || Hkv <= 0 || S_cap < 0 || !(scale > 0.f)) return TV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return TV_ERR_INVALID_ARG;
-  if ((flags & ~(unsigned)TV_ATTN_PREFIX_READY) != 0) return TV_ERR_INVALID_ARG;
+  if ((flags & ~(unsigned)(TV_ATTN_PREFIX_READY | TV_ATTN_ROPE)) != 0) return TV_ERR_INVALID_ARG;
+  const bool rope = (flags & TV_ATTN_ROPE) != 0;
+  if (rope && (!depth || !(rope_theta > 1.0f))) return TV_ERR_INVALID_ARG;
+  if (slot && n_slots < 1) return TV_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
+  if (rope && D != 128) return TV_ERR_UNSUPPORTED;
   if (M + 1 > kMaxRows || S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
   if (B == 0) {
     call.nothing_to_do = true;
@@ -465,8 +474,13 @@ tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t
   p.scale_log2 = scale * 1.4426950408889634f;
   p.flags = flags;
   p.wait_limit_ns = pipeline_wait_limit_ns();
+  p.depth = rope ? depth : nullptr;
+  p.slot = slot;
+  p.n_slots = slot ? n_slots : B;
+  rope_freqs(rope ? (double)rope_theta : 2.0, D, p.rope);
   p.ws = nullptr;
-  if (!encode_kv_map(&call.tmk, k, B * Hkv, S_cap, D) || !encode_kv_map(&call.tmv, v, B * Hkv, S_cap, D))
+  if ((int64_t)p.n_slots * Hkv > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
+  if (!encode_kv_map(&call.tmk, k, p.n_slots * Hkv, S_cap, D) || !encode_kv_map(&call.tmv, v, p.n_slots * Hkv, S_cap, D))
     return TV_ERR_INVALID_ARG;
   if (D == 128) return plan_attention_tc(B, M, Hq, Hkv, S_cap, call.plan);
   return TV_OK;
@@ -492,11 +506,12 @@ extern "C" tv_status tree_attention(const uint16_t* q, const uint16_t* k, const 
                                     const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                                     int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale,
                                     uint16_t* out, void* workspace, size_t workspace_bytes, unsigned flags,
+                                    const int32_t* depth, float rope_theta, const int32_t* slot, int n_slots,
                                     tv_stream_t stream) {
   using namespace tv;
   AttnCall call;
   tv_status r = prepare_attention(q, k, v, S_cap, kv_start, kv_len, anc_mask, status, B, M, Hq, Hkv, D, scale,
-                                  out, flags, call);
+                                  out, flags, depth, rope_theta, slot, n_slots, call);
   if (r != TV_OK || call.nothing_to_do) return r;
   if (D == 128 && call.plan.ws_bytes > 0) {
     if (!workspace || workspace_bytes < call.plan.ws_bytes || !aligned16(workspace)) return TV_ERR_INVALID_ARG;
@@ -558,7 +573,7 @@ extern "C" tv_status tree_attention_noalloc(const uint16_t* q, const uint16_t* k
   using namespace tv;
   AttnCall call;
   tv_status r = prepare_attention(q, k, v, S_cap, kv_start, kv_len, anc_mask, status, B, M, Hq, Hkv, D, scale,
-                                  out, 0u, call);
+                                  out, 0u, nullptr, 0.f, nullptr, 0, call);
   if (r != TV_OK || call.nothing_to_do) return r;
   if (D == 128 && call.plan.ws_bytes > 0) {  // D = 64 keeps its partials on chip
     if (call.plan.ws_bytes > kNoAllocScratchBytes) return TV_ERR_UNSUPPORTED;  // too large for the fixed scratch

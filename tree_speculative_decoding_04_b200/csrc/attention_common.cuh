@@ -27,6 +27,10 @@ struct AttnParams {
   int v_stages;         // V ring depth of the tensor-core kernel
   float scale_log2;     // softmax scale * log2(e)
   unsigned flags;       // TV_ATTN_* launch flags
+  const int32_t* depth; // [B][M+1] node depths (rotary positions kv_len + depth), TV_ATTN_ROPE only
+  const int32_t* slot;  // [B] cache slot of each batch row, or null (slot = row)
+  int n_slots;          // slots of the cache pool (B without a slot map)
+  RopeFreqs rope;       // inverse frequencies, TV_ATTN_ROPE only
   uint64_t wait_limit_ns;  // limit of the pipeline waits (the drain waits keep kWaitLimitNs)
   float* ws;            // split partials: [units][nsplit][128 rows][128] O, then [units][nsplit][128][2] (m, l)
 };
@@ -83,7 +87,8 @@ struct AttnCall {
 tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t S_cap,
                             const int32_t* kv_start, const int32_t* kv_len, const uint32_t* anc_mask,
                             int32_t* status, int B, int M, int Hq, int Hkv, int D, float scale, uint16_t* out,
-                            unsigned flags, AttnCall& call);
+                            unsigned flags, const int32_t* depth, float rope_theta, const int32_t* slot,
+                            int n_slots, AttnCall& call);
 tv_status launch_attention(AttnCall& call, int D, cudaStream_t s);
 
 }  // namespace tv

@@ -219,19 +219,20 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
-  auto issue_k = [&](int i, int32_t ks_, int k_lo_) {
+  // zc_: the tensor-map row block of (cache slot, kv head)
+  auto issue_k = [&](int i, int32_t ks_, int k_lo_, int zc_) {
     const int s = i % k_stages;
     uint8_t* dst = k_ring + s * kTileBytes;
     mbar_arrive_expect_tx(&sh->k_full[s], kTileBytes);
-    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks_ + k_lo_ + i * kKeyTile, bh);
-    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks_ + k_lo_ + i * kKeyTile, bh);
+    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks_ + k_lo_ + i * kKeyTile, zc_);
+    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks_ + k_lo_ + i * kKeyTile, zc_);
   };
-  auto issue_v = [&](int i, int32_t ks_, int k_lo_) {
+  auto issue_v = [&](int i, int32_t ks_, int k_lo_, int zc_) {
     const int s = i % v_stages;
     uint8_t* dst = v_ring + s * kTileBytes;
     mbar_arrive_expect_tx(&sh->v_full[s], kTileBytes);
-    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks_ + k_lo_ + i * kKeyTile, bh);
-    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks_ + k_lo_ + i * kKeyTile, bh);
+    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks_ + k_lo_ + i * kKeyTile, zc_);
+    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks_ + k_lo_ + i * kKeyTile, zc_);
   };
   // This sequence's key tiles are dealt evenly over the splits (ragged batches
   // would otherwise leave short sequences in one split).
@@ -244,8 +245,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   // With programmatic launch this CTA can be resident while the previous kernel
   // is still finishing.
   //  - TV_ATTN_PREFIX_READY: the caller guarantees that the previous launch on
-  //    the stream writes neither the geometry nor any prefix column, so the
-  //    geometry is read now and the first ring's worth of tiles that lie wholly
+  //    the stream writes neither the geometry, the slot map nor any prefix
+  //    column, so the geometry is read now and the first ring's worth of tiles that lie wholly
   //    inside the prefix is requested into shared memory before the grid
   //    dependency resolves.  Tiles reaching the tree rows, the query rows, the
   //    ancestor rows and the status are read only after it.
@@ -260,11 +261,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   // before the CTA exits always keep the full limit
   const uint64_t lim = p.wait_limit_ns;
   int32_t ks = 0, kl = 0;
+  int sl = -1;                 // cache slot of this batch row (-1: outside the pool)
   int npre_k = 0, npre_v = 0;  // tiles requested before the grid dependency
   if (prefix_ready) {
-    ks = __ldcg(p.kv_start + b);
-    kl = __ldcg(p.kv_len + b);
-    if (aligned_ok && geometry_ok(ks, kl, p.M, p.S_cap)) {
+    sl = cache_slot(p.slot, b, p.n_slots);
+    if (sl >= 0) {
+      ks = __ldcg(p.kv_start + sl);
+      kl = __ldcg(p.kv_len + sl);
+    }
+    if (sl >= 0 && aligned_ok && geometry_ok(ks, kl, p.M, p.S_cap)) {
       int k_lo_pre, nt_pre;
       split_range(kl, k_lo_pre, nt_pre);
       const int n_prefix = max(0, min(nt_pre, (kl - k_lo_pre) / kKeyTile));  // tiles wholly inside the prefix
@@ -272,22 +277,25 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       npre_v = min(n_prefix, v_stages);
       if (warp == 0 && lane == 0)  // the thread that initialised the barriers
         for (int i = 0; i < max(npre_k, npre_v); ++i) {
-          if (i < npre_k) issue_k(i, ks, k_lo_pre);
-          if (i < npre_v) issue_v(i, ks, k_lo_pre);
+          if (i < npre_k) issue_k(i, ks, k_lo_pre, sl * p.Hkv + hk);
+          if (i < npre_v) issue_v(i, ks, k_lo_pre, sl * p.Hkv + hk);
         }
     }
   } else if (warp == 0 && lane == 0) {
-    const int32_t ks_h = __ldcg(p.kv_start + b), kl_h = __ldcg(p.kv_len + b);
-    if (geometry_ok(ks_h, kl_h, p.M, p.S_cap)) {
-      int k_lo_h, nt_h;
-      split_range(kl_h, k_lo_h, nt_h);
-      const int nt = min(kPrefetchTiles, nt_h);
-      for (int i = 0; i < nt; ++i) {
-        const int row = ks_h + k_lo_h + i * kKeyTile;
-        tma_prefetch_3d(&tmk, 0, row, bh);
-        tma_prefetch_3d(&tmk, 64, row, bh);
-        tma_prefetch_3d(&tmv, 0, row, bh);
-        tma_prefetch_3d(&tmv, 64, row, bh);
+    const int sl_h = p.slot ? __ldcg(p.slot + b) : b;
+    if (sl_h >= 0 && sl_h < p.n_slots) {
+      const int32_t ks_h = __ldcg(p.kv_start + sl_h), kl_h = __ldcg(p.kv_len + sl_h);
+      if (geometry_ok(ks_h, kl_h, p.M, p.S_cap)) {
+        int k_lo_h, nt_h;
+        split_range(kl_h, k_lo_h, nt_h);
+        const int nt = min(kPrefetchTiles, nt_h);
+        for (int i = 0; i < nt; ++i) {
+          const int row = ks_h + k_lo_h + i * kKeyTile;
+          tma_prefetch_3d(&tmk, 0, row, sl_h * p.Hkv + hk);
+          tma_prefetch_3d(&tmk, 64, row, sl_h * p.Hkv + hk);
+          tma_prefetch_3d(&tmv, 0, row, sl_h * p.Hkv + hk);
+          tma_prefetch_3d(&tmv, 64, row, sl_h * p.Hkv + hk);
+        }
       }
     }
   }
@@ -301,14 +309,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   }
   pdl_wait_primary();
   pdl_launch_dependents();
-  // The geometry is read again after the dependency: if the caller's promise
-  // did not hold (it changed), the sequence is flagged instead of computed.
-  const int32_t ks_now = p.kv_start[b], kl_now = p.kv_len[b];
-  const bool broken_promise = prefix_ready && (ks_now != ks || kl_now != kl);
+  // The slot and the geometry are read again after the dependency: if the
+  // caller's promise did not hold (they changed), the sequence is flagged
+  // instead of computed.
+  const int sl_now = cache_slot(p.slot, b, p.n_slots);
+  const int32_t ks_now = sl_now >= 0 ? p.kv_start[sl_now] : 0, kl_now = sl_now >= 0 ? p.kv_len[sl_now] : 0;
+  const bool broken_promise = prefix_ready && (sl_now != sl || ks_now != ks || kl_now != kl);
+  sl = sl_now;
   ks = ks_now;
   kl = kl_now;
-  const bool valid =
-      aligned_ok && !broken_promise && p.status[b] == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
+  const int zc = sl * p.Hkv + hk;  // tensor-map row block of this (slot, kv head)
+  const bool valid = aligned_ok && sl >= 0 && !broken_promise && p.status[b] == 0 &&
+                     geometry_ok(ks, kl, p.M, p.S_cap);
   const int N = kl + p.M + 1;
   int k_lo = 0, nt_geo = 0;
   split_range(kl, k_lo, nt_geo);
@@ -319,8 +331,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   // overlaps the set-up.
   if (warp == 0 && lane == 0)
     for (int i = 0; i < min(ntiles, max(k_stages, v_stages)); ++i) {
-      if (i < k_stages && i >= npre_k) issue_k(i, ks, k_lo);
-      if (i < v_stages && i >= npre_v) issue_v(i, ks, k_lo);
+      if (i < k_stages && i >= npre_k) issue_k(i, ks, k_lo, zc);
+      if (i < v_stages && i >= npre_v) issue_v(i, ks, k_lo, zc);
     }
   const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
   const int gr = qtile * kRows + r;
@@ -329,13 +341,22 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   const int u = min(gr / p.G, p.M);
   uint32_t anc_w[kMaxRows / 32];
   if (warp >= 2) {
-    // Q row -> swizzled smem (two 64-column boxes); rows past the tile are zero
+    // Q row -> swizzled smem (two 64-column boxes); rows past the tile are zero.
+    // With TV_ATTN_ROPE the row is rotated to its tree position kv_len +
+    // depth(u) on the way (pairs (i, i + 64) sit in chunks c and c + 8).
     const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * (p.M + 1) + u) * p.Hq + hq) * 128);
+    const bool rope = (p.flags & TV_ATTN_ROPE) != 0;
+    const int pos = (rope && row_ok) ? kl + p.depth[(int64_t)b * (p.M + 1) + u] : 0;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (row_ok) v = __ldg(src + c);
-      *reinterpret_cast<uint4*>(q_s + (c >> 3) * (kRows * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+    for (int c = 0; c < 8; ++c) {
+      uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+      if (row_ok) {
+        lo = __ldg(src + c);
+        hi = __ldg(src + c + 8);
+        if (rope) rope_rotate8(lo, hi, pos, p.rope.f, 8 * c);
+      }
+      *reinterpret_cast<uint4*>(q_s + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
+      *reinterpret_cast<uint4*>(q_s + kRows * 128 + r * 128 + ((c ^ (r & 7)) << 4)) = hi;
     }
     fence_async_smem();  // generic-proxy stores -> visible to the tensor core after the barrier
 #pragma unroll
@@ -369,7 +390,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
             to = true;
             break;
           }
-          issue_k(i, ks, k_lo);
+          issue_k(i, ks, k_lo, zc);
           ++k_issued;
         }
         if (i >= v_stages) {
@@ -377,7 +398,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
             to = true;
             break;
           }
-          issue_v(i, ks, k_lo);
+          issue_v(i, ks, k_lo, zc);
           ++v_issued;
         }
       }
@@ -684,7 +705,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && (sh->timed_out || !aligned_ok)) atomicOr(&p.status[b], kSeqTimeout);
-  if (threadIdx.x == 0 && broken_promise) atomicOr(&p.status[b], kSeqBadGeometry);
+  if (threadIdx.x == 0 && (broken_promise || sl < 0)) atomicOr(&p.status[b], kSeqBadGeometry);
 }
 
 }  // namespace

@@ -20,6 +20,11 @@
 // the attention mask and position IDs; a one-CTA kernel, launched as a
 // programmatic dependent, publishes the new kv_start / kv_len / max_len after
 // every run has read the old ones.
+//
+// Slot map (optional): batch row b lives in cache slot slot[b] of a pool; the
+// geometry and the mask / position rows belong to the slot, so a batch can be
+// any set of the pool's sequences (cross-batch scheduling, "Batch Speculative
+// Decoding Done Right", section 2, EXSPEC) without moving their caches.
 #include <algorithm>
 
 #include "tv_common.cuh"
@@ -32,18 +37,27 @@ constexpr int kMoveUnroll = 4;  // uint4 per thread per chunk
 constexpr int kPlanThreads = 256;
 
 struct Plan {
-  int good;  // geometry in range
+  int good;  // slot and geometry in range
   int nb;    // committed rows (0 or accept_len + 1)
+  int sl;    // cache slot of the batch row
   int ks, len;
+};
+
+// Slot map: batch row b lives in cache slot slot[b] (slot == null: slot b);
+// the geometry arrays and the mask / position rows are indexed by slot.
+struct Slots {
+  const int32_t* slot;
+  int n;
 };
 
 __device__ __forceinline__ Plan seq_plan(int b, int M, int64_t S_cap, int max_depth, const int32_t* path,
                                          const int32_t* accept_len, const int32_t* status, const int32_t* kv_start,
-                                         const int32_t* kv_len) {
+                                         const int32_t* kv_len, Slots slots) {
   Plan p;
-  p.ks = kv_start[b];
-  p.len = kv_len[b];
-  p.good = geometry_ok(p.ks, p.len, M, S_cap) ? 1 : 0;
+  p.sl = cache_slot(slots.slot, b, slots.n);
+  p.ks = p.sl >= 0 ? kv_start[p.sl] : 0;
+  p.len = p.sl >= 0 ? kv_len[p.sl] : 0;
+  p.good = (p.sl >= 0 && geometry_ok(p.ks, p.len, M, S_cap)) ? 1 : 0;
   const int a = accept_len[b];
   int nb = 0;
   if (p.good && status[b] == 0 && a >= 0 && a <= max_depth && a <= M) {
@@ -64,10 +78,10 @@ __device__ __forceinline__ Plan seq_plan(int b, int M, int64_t S_cap, int max_de
 // Lmax' over the batch (block-wide reduction; every thread gets the result).
 __device__ int batch_new_max(int B, int M, int64_t S_cap, int max_depth, int realign, const int32_t* path,
                              const int32_t* accept_len, const int32_t* status, const int32_t* kv_start,
-                             const int32_t* kv_len, int* red) {
+                             const int32_t* kv_len, Slots slots, int* red) {
   int mx = 0;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const Plan p = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len);
+    const Plan p = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len, slots);
     if (p.good) mx = max(mx, realign ? p.len + p.nb : p.ks + p.len + p.nb);
   }
 #pragma unroll
@@ -87,7 +101,7 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
     int64_t S_cap, int M, const int32_t* __restrict__ path, const int32_t* __restrict__ accept_len,
     const int32_t* __restrict__ status, int max_depth, const int32_t* __restrict__ kv_start,
     const int32_t* __restrict__ kv_len, int realign, int64_t runs, uint8_t* __restrict__ attn_mask,
-    int32_t* __restrict__ pos_ids) {
+    int32_t* __restrict__ pos_ids, Slots slots) {
   pdl_wait_primary();
   pdl_launch_dependents();
   extern __shared__ uint4 tail[];  // [max_depth + 1][D / 8]
@@ -99,18 +113,20 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
   } else {
     b = (int)((run / Hkv) % B);
   }
-  const Plan me = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len);
+  const Plan me = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len, slots);
   int new_start = me.ks;
   if (realign) {
-    const int lmax = batch_new_max(B, M, S_cap, max_depth, realign, path, accept_len, status, kv_start, kv_len, red);
+    const int lmax =
+        batch_new_max(B, M, S_cap, max_depth, realign, path, accept_len, status, kv_start, kv_len, slots, red);
     new_start = lmax - (me.len + me.nb);
   }
-  if (run >= runs) {  // mask / position-ID row of sequence b
+  if (run >= runs) {  // mask / position-ID row of sequence b (row of its slot)
+    if (me.sl < 0) return;
     const int lo = new_start, hi = new_start + me.len + me.nb;
     for (int64_t t = threadIdx.x; t < S_cap; t += blockDim.x) {
       const bool in = me.good && t >= lo && t < hi;
-      if (attn_mask) attn_mask[(int64_t)b * S_cap + t] = in ? 1 : 0;
-      if (pos_ids) pos_ids[(int64_t)b * S_cap + t] = in ? (int32_t)(t - lo) : 0;
+      if (attn_mask) attn_mask[(int64_t)me.sl * S_cap + t] = in ? 1 : 0;
+      if (pos_ids) pos_ids[(int64_t)me.sl * S_cap + t] = in ? (int32_t)(t - lo) : 0;
     }
     return;
   }
@@ -122,7 +138,7 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
   const int layer = (int)(run / ((int64_t)Hkv * B * 2));
   uint16_t* base = (kvsel ? v_layers : k_layers)[layer];
   const int RV = D >> 3;  // uint4 per row
-  uint4* cache = reinterpret_cast<uint4*>(base + ((int64_t)b * Hkv + h) * S_cap * D);
+  uint4* cache = reinterpret_cast<uint4*>(base + ((int64_t)me.sl * Hkv + h) * S_cap * D);
   const int32_t* pb = path + (int64_t)b * (max_depth + 1);
 
   // (1) stage the committed tail rows (all of them are read before any store)
@@ -187,20 +203,21 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
 __global__ void __launch_bounds__(kPlanThreads) kv_finalize_kernel(
     int B, int M, int64_t S_cap, int max_depth, int realign, const int32_t* __restrict__ path,
     const int32_t* __restrict__ accept_len, int32_t* __restrict__ status, int32_t* __restrict__ kv_start,
-    int32_t* __restrict__ kv_len, int32_t* __restrict__ max_len) {
+    int32_t* __restrict__ kv_len, int32_t* __restrict__ max_len, Slots slots) {
   __shared__ int red[kPlanThreads / 32];
   pdl_wait_primary();
   pdl_launch_dependents();
-  const int lmax = batch_new_max(B, M, S_cap, max_depth, realign, path, accept_len, status, kv_start, kv_len, red);
+  const int lmax =
+      batch_new_max(B, M, S_cap, max_depth, realign, path, accept_len, status, kv_start, kv_len, slots, red);
   // every thread finished reading the old values inside batch_new_max (it ends with a barrier)
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
-    const Plan p = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len);
+    const Plan p = seq_plan(b, M, S_cap, max_depth, path, accept_len, status, kv_start, kv_len, slots);
     if (!p.good) {
       status[b] |= kSeqBadGeometry;
       continue;
     }
-    kv_len[b] = p.len + p.nb;
-    kv_start[b] = realign ? lmax - (p.len + p.nb) : p.ks;
+    kv_len[p.sl] = p.len + p.nb;
+    kv_start[p.sl] = realign ? lmax - (p.len + p.nb) : p.ks;
   }
   if (threadIdx.x == 0) *max_len = lmax;
 }
@@ -212,10 +229,12 @@ extern "C" tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* cons
                                        int D, int64_t S_cap, int M, const int32_t* path, const int32_t* accept_len,
                                        int32_t* status, int max_depth, int32_t* kv_start, int32_t* kv_len,
                                        int32_t* max_len, int realign, uint8_t* attn_mask, int32_t* pos_ids,
-                                       tv_stream_t stream) {
+                                       const int32_t* slot, int n_slots, tv_stream_t stream) {
   using namespace tv;
   if (L < 0 || B < 0 || Hkv < 0 || M < 0 || max_depth < 0 || S_cap < 0 || (realign != 0 && realign != 1))
     return TV_ERR_INVALID_ARG;
+  if (slot && n_slots < 1) return TV_ERR_INVALID_ARG;
+  const Slots slots{slot, slot ? n_slots : B};
   if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
   if (M + 1 > kMaxRows || max_depth + 1 > kMaxRows) return TV_ERR_UNSUPPORTED;
   if (S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
@@ -231,9 +250,9 @@ extern "C" tv_status kv_commit_realign(uint16_t* const* k_layers, uint16_t* cons
     if (e != cudaSuccess) return record_cuda_error(e);
     tv_status r = launch(kv_move_kernel, dim3((unsigned)(runs + extra)), dim3(kMoveThreads), smem, s, 1, true,
                          k_layers, v_layers, B, Hkv, D, S_cap, M, path, accept_len, (const int32_t*)status, max_depth,
-                         (const int32_t*)kv_start, (const int32_t*)kv_len, realign, runs, attn_mask, pos_ids);
+                         (const int32_t*)kv_start, (const int32_t*)kv_len, realign, runs, attn_mask, pos_ids, slots);
     if (r != TV_OK) return r;
   }
   return launch(kv_finalize_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1, true, B, M, S_cap, max_depth,
-                realign, path, accept_len, status, kv_start, kv_len, max_len);
+                realign, path, accept_len, status, kv_start, kv_len, max_len, slots);
 }

@@ -11,6 +11,14 @@
 // order, 16 bytes per thread and access, a few accesses in flight per thread
 // (all loads of a batch before its stores); each destination row is D * 2
 // contiguous bytes.  The grid is a multiple of the SM count, grid-stride.
+//
+// Rotary position embedding (optional): the K rows are rotated to their tree
+// position kv_len + depth (position-ID contiguity, "Batch Speculative Decoding
+// Done Right", section 2) on the way into the cache, so the committed cache
+// holds rotated keys as the attention expects; V rows are copied as they are.
+//
+// Slot map (optional): batch row b writes into cache slot slot[b] of a pool of
+// n_slots sequences, whose geometry is kv_start[slot[b]], kv_len[slot[b]].
 #include <algorithm>
 
 #include "tv_common.cuh"
@@ -21,14 +29,51 @@ namespace {
 constexpr int kWriteThreads = 256;
 constexpr int kWriteUnroll = 4;
 
-__global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
-    uint16_t* const* __restrict__ k_layers, uint16_t* const* __restrict__ v_layers,
-    const uint4* __restrict__ tree_k, const uint4* __restrict__ tree_v, int B, int Hkv, int RV, int64_t S_cap,
-    int M, const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len, int64_t per_kv) {
+// Rotary variant of the K rows: one work item per pair of 16-byte chunks (c,
+// c + RV/2) of a K row, rotated to position kv_len + depth[b][r].
+__global__ void __launch_bounds__(kWriteThreads) kv_write_rope_k_kernel(
+    uint16_t* const* __restrict__ k_layers, const uint4* __restrict__ tree_k, int B, int Hkv, int RV,
+    int64_t S_cap, int M, const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len,
+    const int32_t* __restrict__ depth, const int32_t* __restrict__ slot, int n_slots, int64_t items,
+    const __grid_constant__ RopeFreqs fr) {
   pdl_wait_primary();
   pdl_launch_dependents();
   const int n = M + 1;
-  const int64_t total = 2 * per_kv;  // 16-byte units: K then V
+  const int half = RV / 2;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < items; w += stride) {
+    const int c = (int)(w % half);
+    const int64_t row = w / half;  // ((l * B + b) * Hkv + h) * n + r
+    const int r = (int)(row % n);
+    const int64_t run = row / n;
+    const int h = (int)(run % Hkv);
+    const int64_t lb = run / Hkv;
+    const int b = (int)(lb % B);
+    const int l = (int)(lb / B);
+    const int sl = cache_slot(slot, b, n_slots);
+    if (sl < 0) continue;
+    const int32_t ks = kv_start[sl], kl = kv_len[sl];
+    if (!geometry_ok(ks, kl, M, S_cap)) continue;
+    uint4 lo = tree_k[row * RV + c], hi = tree_k[row * RV + c + half];
+    rope_rotate8(lo, hi, kl + depth[(int64_t)b * n + r], fr.f, 8 * c);
+    uint4* cache = reinterpret_cast<uint4*>(k_layers[l]) + (((int64_t)sl * Hkv + h) * S_cap + ks + kl + r) * RV;
+    cache[c] = lo;
+    cache[c + half] = hi;
+  }
+}
+
+// kv = 0: K and V rows (plain copy); kv = 1 only V rows (the K rows are
+// written by the rotary kernel).
+__global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
+    uint16_t* const* __restrict__ k_layers, uint16_t* const* __restrict__ v_layers,
+    const uint4* __restrict__ tree_k, const uint4* __restrict__ tree_v, int B, int Hkv, int RV, int64_t S_cap,
+    int M, const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len,
+    const int32_t* __restrict__ slot, int n_slots, int64_t per_kv, int v_only) {
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  const int n = M + 1;
+  const int64_t first = v_only ? per_kv : 0;
+  const int64_t total = 2 * per_kv - first;  // 16-byte units: K then V
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
        base += stride * kWriteUnroll) {
@@ -37,8 +82,8 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
 #pragma unroll
     for (int t = 0; t < kWriteUnroll; ++t) {
       dst[t] = nullptr;
-      const int64_t u = base + (int64_t)t * stride;
-      if (u >= total) continue;
+      const int64_t u = first + base + (int64_t)t * stride;
+      if (u >= 2 * per_kv) continue;
       const int kv = u >= per_kv;
       const int64_t w = kv ? u - per_kv : u;  // index inside [L][B][Hkv][n][RV]
       const int c = (int)(w % RV);
@@ -49,11 +94,13 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
       const int64_t lb = run / Hkv;
       const int b = (int)(lb % B);
       const int l = (int)(lb / B);
-      const int32_t ks = kv_start[b], kl = kv_len[b];
+      const int sl = cache_slot(slot, b, n_slots);
+      if (sl < 0) continue;
+      const int32_t ks = kv_start[sl], kl = kv_len[sl];
       if (!geometry_ok(ks, kl, M, S_cap)) continue;
       val[t] = kv ? tree_v[w] : tree_k[w];
       uint4* cache = reinterpret_cast<uint4*>((kv ? v_layers : k_layers)[l]);
-      dst[t] = cache + (((int64_t)b * Hkv + h) * S_cap + ks + kl + r) * RV + c;
+      dst[t] = cache + (((int64_t)sl * Hkv + h) * S_cap + ks + kl + r) * RV + c;
     }
 #pragma unroll
     for (int t = 0; t < kWriteUnroll; ++t)
@@ -66,12 +113,16 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
 
 extern "C" tv_status tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v_layers, const uint16_t* tree_k,
                                    const uint16_t* tree_v, int L, int B, int Hkv, int D, int64_t S_cap, int M,
-                                   const int32_t* kv_start, const int32_t* kv_len, tv_stream_t stream) {
+                                   const int32_t* kv_start, const int32_t* kv_len, const int32_t* depth,
+                                   float rope_theta, const int32_t* slot, int n_slots, tv_stream_t stream) {
   using namespace tv;
   if (L < 0 || B < 0 || Hkv < 0 || M < 0 || S_cap < 0) return TV_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return TV_ERR_UNSUPPORTED;
   if (M + 1 > kMaxRows) return TV_ERR_UNSUPPORTED;
   if (S_cap > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
+  if (slot && n_slots < 1) return TV_ERR_INVALID_ARG;
+  const bool rope = depth != nullptr;
+  if (rope && !(rope_theta > 1.0f)) return TV_ERR_INVALID_ARG;
   const int64_t per_kv = (int64_t)L * B * Hkv * (M + 1) * (D / 8);
   if (per_kv == 0) return TV_OK;
   if (!k_layers || !v_layers || !tree_k || !tree_v || !kv_start || !kv_len) return TV_ERR_INVALID_ARG;
@@ -80,10 +131,22 @@ extern "C" tv_status tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t need = (2 * per_kv + (int64_t)kWriteThreads * kWriteUnroll - 1) / ((int64_t)kWriteThreads * kWriteUnroll);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (rope) {
+    RopeFreqs fr;
+    rope_freqs((double)rope_theta, D, fr);
+    const int64_t items = per_kv / 2;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((items + kWriteThreads - 1) / kWriteThreads,
+                                                                  (int64_t)sms * 8));
+    tv_status r = launch(kv_write_rope_k_kernel, dim3((unsigned)blocks), dim3(kWriteThreads), 0, s, 1, true,
+                         k_layers, reinterpret_cast<const uint4*>(tree_k), B, Hkv, D / 8, S_cap, M, kv_start, kv_len,
+                         depth, slot, slot ? n_slots : B, items, fr);
+    if (r != TV_OK) return r;
+  }
+  const int64_t units = rope ? per_kv : 2 * per_kv;
+  const int64_t need = (units + (int64_t)kWriteThreads * kWriteUnroll - 1) / ((int64_t)kWriteThreads * kWriteUnroll);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)sms * 8));
-  return launch(kv_write_kernel, dim3((unsigned)blocks), dim3(kWriteThreads), 0,
-                reinterpret_cast<cudaStream_t>(stream), 1, true, k_layers, v_layers,
+  return launch(kv_write_kernel, dim3((unsigned)blocks), dim3(kWriteThreads), 0, s, 1, true, k_layers, v_layers,
                 reinterpret_cast<const uint4*>(tree_k), reinterpret_cast<const uint4*>(tree_v), B, Hkv, D / 8, S_cap,
-                M, kv_start, kv_len, per_kv);
+                M, kv_start, kv_len, slot, slot ? n_slots : B, per_kv, rope ? 1 : 0);
 }

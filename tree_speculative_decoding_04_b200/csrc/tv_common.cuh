@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda.h>  // CUtensorMap and driver enums (types only; the driver is reached through the runtime)
+#include <math.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -25,6 +26,26 @@ constexpr uint32_t kWaitLimitPolls = 1u << 28;
 
 __host__ __device__ inline bool geometry_ok(int32_t ks, int32_t kl, int M, int64_t S_cap) {
   return ks >= 0 && kl >= 0 && (int64_t)ks + kl + M + 1 <= S_cap;
+}
+
+// Largest head dim with a rotary table: D / 2 angle frequencies.
+constexpr int kMaxRopePairs = 64;
+
+// Inverse frequencies theta^(-2i/D), i < D/2, computed on the host in double.
+struct RopeFreqs {
+  double f[kMaxRopePairs];
+};
+
+inline void rope_freqs(double theta, int D, RopeFreqs& r) {
+  for (int i = 0; i < kMaxRopePairs; ++i) r.f[i] = i < D / 2 ? pow(theta, -2.0 * i / D) : 0.0;
+}
+
+// Cache slot of batch row b: slot[b] when a slot map is given, else b; -1 if
+// the map points outside [0, n_slots).
+__host__ __device__ inline int cache_slot(const int32_t* slot, int b, int n_slots) {
+  if (!slot) return b;
+  const int s = slot[b];
+  return (s >= 0 && s < n_slots) ? s : -1;
 }
 
 #if defined(__CUDACC__)
@@ -144,6 +165,37 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------------- rotary embedding
+// cos and sin of the angle pos * inv_freq.  The angle is formed and reduced to
+// [-pi, pi] in double precision (two-part 2 pi, Cody-Waite style), so that the
+// single-precision sine and cosine see an argument accurate to float rounding
+// even at positions of tens of thousands.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
+  const double a = (double)pos * inv_freq;
+  const double k = rint(a * 0.15915494309189535);   // a / (2 pi), nearest integer
+  double r = fma(-k, 6.283185307179586, a);         // 2 pi, leading double
+  r = fma(-k, 2.4492935982947064e-16, r);           // 2 pi, remainder
+  sincosf((float)r, &s, &c);
+}
+
+// Rotate 8 pairs: lo holds elements i0 .. i0+7 of a row, hi the elements
+// i0 + D/2 .. i0 + D/2 + 7; pair (x, y) becomes (x cos - y sin, y cos + x sin),
+// rounded to bf16.
+__device__ __forceinline__ void rope_rotate8(uint4& lo, uint4& hi, int pos, const double* inv_freq, int i0) {
+  uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* h = reinterpret_cast<uint32_t*>(&hi);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&l[w]));
+    const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h[w]));
+    float c0, s0, c1, s1;
+    rope_cos_sin(pos, inv_freq[i0 + 2 * w], c0, s0);
+    rope_cos_sin(pos, inv_freq[i0 + 2 * w + 1], c1, s1);
+    l[w] = pack_bf16x2(fmaf(x.x, c0, -y.x * s0), fmaf(x.y, c1, -y.y * s1));
+    h[w] = pack_bf16x2(fmaf(y.x, c0, x.x * s0), fmaf(y.y, c1, x.y * s1));
+  }
 }
 
 #endif  // __CUDACC__

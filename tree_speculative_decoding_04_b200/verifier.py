@@ -78,12 +78,16 @@ class StepResult:
 
 class TreeVerifier:
     def __init__(self, B, M, Hq, Hkv, D, V, L, S_cap, max_depth, realign=False, device="cuda",
-                 k_layers=None, v_layers=None, with_mask_outputs=None, commit_layers=None):
+                 k_layers=None, v_layers=None, with_mask_outputs=None, commit_layers=None, rope_theta=0.0):
         """k_layers / v_layers: the L per-layer caches (default: allocated here).
         commit_layers: the indices of the layers kv_commit_realign moves (default
-        all); a caller whose layer list repeats a buffer commits each buffer once."""
+        all); a caller whose layer list repeats a buffer commits each buffer once.
+        rope_theta > 0: q and the tree rows' K are given before their rotary
+        embedding; the kernels rotate them to the tree positions kv_len + depth
+        (tree_kv_write for K, tree_attention's query staging for q)."""
         self.B, self.M, self.Hq, self.Hkv, self.D, self.V, self.L = B, M, Hq, Hkv, D, V, L
         self.S_cap, self.max_depth, self.realign = S_cap, max_depth, bool(realign)
+        self.rope_theta = float(rope_theta)
         self.n = M + 1
         self.W = (self.n + 31) // 32
         dev = torch.device(device)
@@ -141,15 +145,17 @@ class TreeVerifier:
         (true after tree_build_mask, tree_kv_write and the attention of another
         layer; false after kv_commit_realign), so prefix tiles may stream while
         it finishes."""
+        flags = (tv.ATTN_PREFIX_READY if prefix_ready else 0) | (tv.ATTN_ROPE if self.rope_theta > 0 else 0)
         tv.tree_attention(self.q[layer], self.k[layer], self.v[layer], self.kv_start, self.kv_len, self.anc,
-                          self.status, self.out[layer], self.workspace, stream=stream,
-                          flags=tv.ATTN_PREFIX_READY if prefix_ready else 0)
+                          self.status, self.out[layer], self.workspace, stream=stream, flags=flags,
+                          depth=self.depth, rope_theta=self.rope_theta)
 
     def write_tree_rows(self, layer, stream=None):
         """tree_k / tree_v of one layer -> the cache, behind each sequence's prefix."""
         tv.tree_kv_write(self.k_ptrs[layer:layer + 1], self.v_ptrs[layer:layer + 1],
                          self.tree_k[layer].unsqueeze(0), self.tree_v[layer].unsqueeze(0), self.S_cap,
-                         self.kv_start, self.kv_len, stream)
+                         self.kv_start, self.kv_len, stream,
+                         depth=self.depth if self.rope_theta > 0 else None, rope_theta=self.rope_theta)
 
     def accept(self, stream=None):
         tv.tree_accept(self.logits, self.draft, self.parent, self.depth, self.anc, self.status, self.max_depth,
