@@ -275,3 +275,79 @@ def round_bf16(x):
     out = np.zeros(x.shape, np.uint16)
     lib().oracle_round_bf16(_p(x), x.size, _p(out))
     return out
+
+
+# ----------------------------------------------------------------------------- cache-slot pools
+# "Batch Speculative Decoding Done Right", methodology: EXSPEC keeps a pool of
+# sequences and batches any of them together (same-length groups need no
+# realignment).  With a slot map, batch row b's cache is slot slots[b] of a pool
+# whose layers are [n_slots][Hkv][S_cap][D] and whose geometry is [n_slots].  The
+# pool versions below are the plainest reading of that: gather the batch's
+# slots, run the batch function above unchanged, scatter the result back.  A
+# slot outside [0, n_slots) is skipped and flagged like a bad geometry.
+
+def _valid_slots(slots, n_slots):
+    slots = np.asarray(slots, np.int64)
+    return slots, (slots >= 0) & (slots < n_slots)
+
+
+def pool_tree_kv_write(k_pool, v_pool, slots, tree_k, tree_v, kv_start, kv_len, depth=None, rope_base: float = 0.0):
+    """tree_kv_write on the batch rows' slots of a pool (in place)."""
+    n_slots = k_pool[0].shape[0]
+    slots, ok = _valid_slots(slots, n_slots)
+    idx = np.nonzero(ok)[0]
+    if len(idx) == 0:
+        return
+    s = slots[idx]
+    kb = [np.ascontiguousarray(k[s]) for k in k_pool]
+    vb = [np.ascontiguousarray(v[s]) for v in v_pool]
+    tree_kv_write(kb, vb, np.asarray(tree_k)[:, idx], np.asarray(tree_v)[:, idx], np.asarray(kv_start)[s],
+                  np.asarray(kv_len)[s], None if depth is None else np.asarray(depth)[idx], rope_base)
+    for layer in range(len(k_pool)):
+        k_pool[layer][s] = kb[layer]
+        v_pool[layer][s] = vb[layer]
+
+
+def pool_tree_attention(q, k_pool, v_pool, slots, kv_start, kv_len, parent, status, Hkv: int,
+                        rope_base: float = 0.0):
+    """tree_attention with batch row b reading cache slot slots[b]; rows whose slot
+    is outside the pool are zero."""
+    n_slots = k_pool.shape[0]
+    slots, ok = _valid_slots(slots, n_slots)
+    st = np.asarray(status, np.int32).copy()
+    st[~ok] |= BAD_GEOMETRY
+    s = np.where(ok, slots, 0)
+    return tree_attention(q, np.ascontiguousarray(k_pool[s]), np.ascontiguousarray(v_pool[s]),
+                          np.asarray(kv_start)[s], np.asarray(kv_len)[s], parent, st, Hkv, rope_base=rope_base)
+
+
+def pool_kv_commit_realign(k_pool, v_pool, slots, M: int, path, accept_len, status, max_depth: int, kv_start, kv_len,
+                           realign: int, attn_mask=None, pos_ids=None):
+    """kv_commit_realign of a batch of pool slots, in place on the pool layers and
+    on the pool geometry kv_start / kv_len ([n_slots], int32, modified).  Returns
+    (max_len, status') ; attn_mask / pos_ids ([n_slots][S_cap]) rows of the
+    batch's slots are rewritten when given."""
+    n_slots = k_pool[0].shape[0]
+    slots, ok = _valid_slots(slots, n_slots)
+    st = np.asarray(status, np.int32).copy()
+    st[~ok] |= BAD_GEOMETRY
+    idx = np.nonzero(ok)[0]
+    if len(idx) == 0:
+        return 0, st
+    s = slots[idx]
+    kb = [np.ascontiguousarray(k[s]) for k in k_pool]
+    vb = [np.ascontiguousarray(v[s]) for v in v_pool]
+    ks2, kl2, ml, am, pos, st2 = kv_commit_realign(kb, vb, M, np.asarray(path)[idx], np.asarray(accept_len)[idx],
+                                                   st[idx], max_depth, np.asarray(kv_start)[s],
+                                                   np.asarray(kv_len)[s], realign, with_mask=True, with_status=True)
+    for layer in range(len(k_pool)):
+        k_pool[layer][s] = kb[layer]
+        v_pool[layer][s] = vb[layer]
+    kv_start[s] = ks2
+    kv_len[s] = kl2
+    st[idx] = st2
+    if attn_mask is not None:
+        attn_mask[s] = am
+    if pos_ids is not None:
+        pos_ids[s] = pos
+    return ml, st
