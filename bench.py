@@ -438,6 +438,95 @@ def per_call_times(ver, cfg, stream, reps, reset):
                 kvw_ms=kvw_ms)
 
 
+def commit_modes(ver, cfg, stream, reps, reset, L_phys, al, path, com_ms, kv_start0, kv_len0):
+    """The commit modes of "EAGLE-Pangu", methodology A, timed on B200 over the
+    distinct layers and scaled to the workload's layers:
+    - fast reorder (this library): kv_commit_realign with the step's path --
+      only the new segment moves, in place;
+    - length-based (this library): the same call with every accepted row
+      already in place (a chain accepted in order) -- nothing moves;
+    - branch cache (the pages' prior art, torch copies here): every step clones
+      the committed cache of every layer into a branch cache, and the accepted
+      rows are then copied from the branch back into the main cache;
+    - full path-index reorder (prior art): the whole content is gathered by an
+      index map (prefix in order, then the accepted rows) instead of only the
+      new segment."""
+    import tree_speculative_decoding_04_b200 as tvpkg  # noqa: F401
+
+    scale = cfg.L / L_phys
+    # length-based: the chain path 0..a, every row already in place
+    saved = ver.path.clone()
+    chain = torch.zeros_like(ver.path)
+    for b in range(cfg.B):
+        a = int(al[b])
+        if a >= 0:
+            chain[b, :a + 1] = torch.arange(a + 1, dtype=torch.int32, device=chain.device)
+    ver.path.copy_(chain)
+
+    def commit_only():
+        reset()
+        ver.commit(stream)
+
+    g = capture(commit_only, stream)
+    len_ms = event_time(g.replay, reps, stream)
+    del g
+    ver.path.copy_(saved)
+    g_reset = capture(reset, stream)
+    reset_ms = event_time(g_reset.replay, reps, stream)
+    len_ms = max(len_ms - reset_ms, 1e-6)
+    # branch cache: clone every layer (one scratch layer, rotated), then copy back
+    # the accepted rows of every sequence from the branch
+    kb = [ver.k[i] for i in range(L_phys)]
+    vb = [ver.v[i] for i in range(L_phys)]
+    scratch = torch.empty_like(kb[0])
+    kl = [int(x) for x in kv_len0]  # the geometry before the commit
+    ks = [int(x) for x in kv_start0]
+    n_acc = [int(a) + 1 if a >= 0 else 0 for a in al]
+    src_idx = [torch.as_tensor([ks[b] + kl[b] + int(path[b, j]) for j in range(n_acc[b])], dtype=torch.long,
+                               device=scratch.device) for b in range(cfg.B)]
+    dst_idx = [torch.as_tensor([ks[b] + kl[b] + j for j in range(n_acc[b])], dtype=torch.long,
+                               device=scratch.device) for b in range(cfg.B)]
+
+    def clone_all():
+        for i in range(L_phys):
+            scratch.copy_(kb[i])
+            scratch.copy_(vb[i])
+
+    def commit_back():
+        for i in range(L_phys):
+            for cache in (kb[i], vb[i]):
+                for b in range(cfg.B):
+                    if n_acc[b]:
+                        cache[b].index_copy_(1, dst_idx[b], scratch[b].index_select(1, src_idx[b]))
+
+    def full_reorder():
+        for i in range(L_phys):
+            for cache in (kb[i], vb[i]):
+                for b in range(cfg.B):
+                    idx = torch.cat([torch.arange(ks[b], ks[b] + kl[b], device=scratch.device), src_idx[b]])
+                    scratch[b, :, :len(idx)].copy_(cache[b].index_select(1, idx))
+
+    with torch.cuda.stream(stream):
+        clone_ms = event_time(clone_all, 2, stream)
+        back_ms = event_time(commit_back, 2, stream)
+        full_ms = event_time(full_reorder, 2, stream)
+    del scratch
+    clone_bytes = L_phys * 2 * kb[0].numel() * 2 * 2  # read + write of each layer's K and V
+    branch_ms = (clone_ms + back_ms) * scale
+    return {
+        "layers_measured": L_phys, "scaled_to_layers": cfg.L,
+        "fast_reorder_us": com_ms * scale * 1e3,
+        "length_based_us": len_ms * scale * 1e3,
+        "branch_cache_us": branch_ms * 1e3,
+        "branch_cache_clone_gbs": clone_bytes / (clone_ms * 1e-3) / 1e9,
+        "full_path_index_reorder_us": full_ms * scale * 1e3,
+        "fast_reorder_speedup_vs_branch_cache": branch_ms / (com_ms * scale),
+        "fast_reorder_speedup_vs_full_reorder": full_ms / com_ms,
+        "note": "branch cache and full reorder are the pages' prior art written with torch copies / index ops "
+                "(comparison arms, not this library's path)",
+    }
+
+
 def measure_step(args, cfg, world, device, steps, warmup, with_clock=False, with_e2e=False):
     """Whole-step timing of a single-step workload.  Returns (record, state)."""
     import tree_speculative_decoding_04_b200 as tvpkg
@@ -494,6 +583,8 @@ def measure_step(args, cfg, world, device, steps, warmup, with_clock=False, with
     shift = (ver.kv_start.cpu().numpy() - host["kv_start"]) if cfg.left_padded else np.zeros(cfg.B, np.int64)
 
     t = per_call_times(ver, cfg, stream, max(5, steps // 2), reset)
+    modes = commit_modes(ver, cfg, stream, max(5, steps // 2), reset, L_phys, al, path, t["com_ms"],
+                         host["kv_start"], host["kv_len"]) if cfg.name in ("mha7b", "b32gqa", "stress") else None
     # the commit ran on the distinct layers only: scale its share to every layer
     scale = cfg.L / L_phys
     ms_step = ms_meas + (scale - 1.0) * t["com_ms"]
@@ -524,6 +615,7 @@ def measure_step(args, cfg, world, device, steps, warmup, with_clock=False, with
                          "tree_attention_single_launch": t["attn_single_ms"] * 1e3,
                          "tree_accept": t["acc_ms"] * 1e3, "kv_commit_realign": t["com_ms"] * 1e3,
                          "geometry_reset_copies": t["reset_ms"] * 1e3},
+        "commit_modes": modes,
         "rope": {"attention_per_layer_us": t["attn_rope_ms"] * 1e3 if t["attn_rope_ms"] else None,
                  "attention_plain_per_layer_us": t["attn_ms"] * 1e3,
                  "attention_overhead_frac": t["attn_rope_ms"] / t["attn_ms"] - 1.0 if t["attn_rope_ms"] else None,
@@ -747,6 +839,86 @@ def measure_rounds(args, cfg, world, device, rounds, replays, warmup, with_clock
     return rec, dict(ver=ver, host=host, clk=clk, stream=stream)
 
 
+def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
+    """Cross-batch scheduling (EXSPEC) on the EQSPEC shapes: a pool of n_slots
+    sequences whose prefix lengths come from a few length buckets (drawn from the
+    workload's range), batches of up to B picked every round by SequencePool
+    (equal lengths: no realignment; else the EQSPEC repad), each round with fresh
+    tree rows, q and logits.  The scheduler needs each round's accept lengths, so
+    every round ends with a host synchronisation; device time (CUDA events
+    around each step) and wall time are both reported, with the share of the
+    device time spent in kv_commit_realign beside the EQSPEC figure."""
+    from tree_speculative_decoding_04_b200.pool import FALLBACK, PoolVerifier, SequencePool
+
+    rng = np.random.default_rng(args.seed + 7)
+    g = W.torch_generator(args.seed + 7, device)
+    B, n, L = cfg.B, cfg.M + 1, cfg.L
+    lo, hi = cfg.prefix[1], cfg.prefix[2]
+    bucket_len = rng.integers(lo, hi + 1, size=buckets)
+    lengths0 = np.sort(rng.choice(bucket_len, size=n_slots)).astype(np.int32)
+    S_cap = int(lengths0.max()) + (rounds + 1) * n + 8
+    S_cap = (S_cap + 7) // 8 * 8
+    pv = PoolVerifier(n_slots, B, cfg.M, cfg.Hq, cfg.Hkv, cfg.D, cfg.V, L, S_cap, cfg.max_depth, device=device,
+                      with_mask_outputs=True)
+    for layer in range(L):
+        pv.k[layer].copy_(W.randn_bf16(pv.k[layer].shape, g, device))
+        pv.v[layer].copy_(W.randn_bf16(pv.v[layer].shape, g, device))
+    pv.kv_len.copy_(torch.as_tensor(lengths0))
+    parent = np.stack([W.make_tree(cfg, rng) for _ in range(B)]).astype(np.int32)
+    pv.parent.copy_(torch.as_tensor(parent))
+    pv.q.copy_(W.randn_bf16(pv.q.shape, g, device))
+    pv.tree_k.copy_(W.randn_bf16(pv.tree_k.shape, g, device))
+    pv.tree_v.copy_(W.randn_bf16(pv.tree_v.shape, g, device))
+    lg = W.randn_f32((rounds, B, n, cfg.V), g, device, cfg.logit_sigma)
+    drafts = [torch.as_tensor(W.plant_drafts(lg[r], parent, cfg.p_plant, rng)).to(device) for r in range(rounds)]
+    pool = SequencePool(lengths0, batch=B)
+    stream = torch.cuda.Stream(device)
+    dev_ms, com_ms, wall = 0.0, 0.0, 0.0
+    n_grouped = n_fallback = 0
+    nodes = 0
+    com_by_mode = {"grouped": 0.0, "fallback": 0.0}
+    torch.cuda.synchronize()
+    for r in range(rounds + 2):  # two untimed warm-up rounds
+        t0 = time.perf_counter()
+        slots, mode = pool.next_batch()
+        Bb = len(slots)
+        pv.logits[:Bb].copy_(lg[r % rounds, :Bb])
+        pv.draft[:Bb].copy_(drafts[r % rounds][:Bb])
+        pv.set_slots(slots, stream)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            pv.step(Bb, 1 if mode == FALLBACK else 0, stream, before_commit=lambda: e1.record(stream))
+            e2.record(stream)
+        e2.synchronize()
+        al = pv.accept_len[:Bb].cpu().numpy()
+        pool.commit(slots, al)
+        t1 = time.perf_counter()
+        if r >= 2:
+            wall += t1 - t0
+            dev_ms += e0.elapsed_time(e2)
+            c = e1.elapsed_time(e2)
+            com_ms += c
+            com_by_mode[mode] += c
+            n_grouped += mode != FALLBACK
+            n_fallback += mode == FALLBACK
+            nodes += Bb * cfg.M
+    rec = {
+        "workload": f"exspec: pool of {n_slots} sequences of the eqspec shapes, prefix lengths from {buckets} buckets "
+                    f"of {lo}-{hi}, batches of up to {B}, {rounds} rounds",
+        "nodes_per_s_device": nodes / (dev_ms * 1e-3), "nodes_per_s_wall": nodes / wall,
+        "ms_per_round_device": dev_ms / rounds, "ms_per_round_wall": wall * 1e3 / rounds,
+        "grouped_rounds": n_grouped, "fallback_rounds": n_fallback,
+        "commit_share_of_device_time": com_ms / dev_ms,
+        "commit_ms_per_round": {k: v / max(1, n_grouped if k == "grouped" else n_fallback)
+                                for k, v in com_by_mode.items()},
+        "gpu_launches_per_round": pv.launches_per_step(),
+        "note": "every round ends with a host synchronisation (the scheduler needs the accept lengths)",
+    }
+    del pv, lg, drafts
+    return rec
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 def cpu_oracle_sample(cfg, q, k, v, logits, host, budget_s, rng, layers_cap=None):
@@ -940,6 +1112,15 @@ def run_ours(args, cfg, world, rank, local):
             except Exception as e:  # a secondary workload must not void the headline line
                 per_config[name] = {"error": repr(e)[:300]}
                 torch.cuda.empty_cache()
+        try:
+            per_config["exspec"] = measure_exspec(args, W.CONFIGS["eqspec"], device)
+            if "eqspec" in per_config and "kv_commit" in per_config["eqspec"]:
+                eq = per_config["eqspec"]
+                per_config["exspec"]["eqspec_commit_share"] = (
+                    eq["kv_commit"]["us"] * 1e-3 / eq["ms_per_round"])
+        except Exception as e:
+            per_config["exspec"] = {"error": repr(e)[:300]}
+        free_state({})
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args, cfg, device)

@@ -132,7 +132,15 @@ __global__ void __launch_bounds__(kMoveThreads) kv_move_kernel(
   }
   if (!me.good) return;
   const int shift = new_start - me.ks;
-  if (shift == 0 && me.nb == 0) return;
+  if (shift == 0) {
+    // Nothing moves when every committed row already sits at its place (a
+    // chain accepted in order): the length-based commit of "EAGLE-Pangu",
+    // methodology A -- only kv_len grows, which kv_finalize_kernel publishes.
+    const int32_t* pb = path + (int64_t)b * (max_depth + 1);
+    bool in_place = true;
+    for (int j = 0; j < me.nb; ++j) in_place = in_place && pb[j] == j;
+    if (in_place) return;
+  }
   const int h = (int)(run % Hkv);
   const int kvsel = (int)((run / ((int64_t)Hkv * B)) & 1);
   const int layer = (int)(run / ((int64_t)Hkv * B * 2));

@@ -16,8 +16,6 @@ EQSPEC repad.
 """
 from __future__ import annotations
 
-import dataclasses
-
 import torch
 
 from . import _lib as tv
@@ -89,15 +87,6 @@ class SequencePool:
         self.active[slot] = False
 
 
-@dataclasses.dataclass
-class PoolStepResult:
-    slots: list
-    mode: str
-    accept_len: torch.Tensor
-    path: torch.Tensor
-    bonus: torch.Tensor
-
-
 class PoolVerifier:
     """One verification step of a batch of pool slots, through the C ABI.
 
@@ -161,9 +150,11 @@ class PoolVerifier:
         with torch.cuda.stream(s):
             self.slot[:Bb].copy_(self._slot_host[:Bb], non_blocking=True)
 
-    def step(self, Bb, realign, stream=None):
+    def step(self, Bb, realign, stream=None, before_commit=None):
         """One verification step of the first Bb batch rows (slots set by
-        set_slots); asynchronous on `stream`."""
+        set_slots); asynchronous on `stream`.  before_commit: optional callable
+        run (on the host) between the accept and the commit launches, e.g. to
+        record a CUDA event."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
         sl = self.slot[:Bb]
         tv.tree_build_mask(self.parent[:Bb], self.max_depth, self.anc[:Bb], self.depth[:Bb], self.status[:Bb], s)
@@ -177,6 +168,8 @@ class PoolVerifier:
         tv.tree_accept(self.logits[:Bb], self.draft[:Bb], self.parent[:Bb], self.depth[:Bb], self.anc[:Bb],
                        self.status[:Bb], self.max_depth, self.argmax[:Bb], self.accept_len[:Bb], self.path[:Bb],
                        self.bonus[:Bb], s)
+        if before_commit is not None:
+            before_commit()
         tv.kv_commit_realign(self.k_ptrs, self.v_ptrs, Bb, self.Hkv, self.D, self.S_cap, self.M, self.path[:Bb],
                              self.accept_len[:Bb], self.status[:Bb], self.max_depth, self.kv_start, self.kv_len,
                              self.max_len, int(realign), self.attn_mask, self.pos_ids, s, slot=sl)
