@@ -84,6 +84,8 @@ def lib():
         _lib.oracle_kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P]
         _lib.oracle_tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P, f64]
         _lib.oracle_rope_rows.argtypes = [P, P, i64, i32, f64]
+        _lib.oracle_lm_head_logits.argtypes = [P, P, P, i64, i32, i32, P]
+        _lib.oracle_argmax_rows_f64.argtypes = [P, i64, i32, P]
         _lib.oracle_round_bf16.argtypes = [P, i64, P]
         for f in (
             _lib.oracle_tree_build_mask,
@@ -351,3 +353,29 @@ def pool_kv_commit_realign(k_pool, v_pool, slots, M: int, path, accept_len, stat
     if pos_ids is not None:
         pos_ids[s] = pos
     return ml, st
+
+
+# ----------------------------------------------------------------------------- LM head
+def lm_head_logits(hidden, w, rows=None):
+    """Exact (double) logits of the selected rows: hidden bf16-bits [R][H], w bf16-bits
+    [V][H] -> float64 [len(rows)][V] (all rows by default)."""
+    hidden, w = _bits16(hidden), _bits16(w)
+    H = hidden.shape[-1]
+    hidden = hidden.reshape(-1, H)
+    V = w.shape[0]
+    assert w.shape == (V, H)
+    rows = np.arange(hidden.shape[0], dtype=np.int32) if rows is None else _c(rows, np.int32)
+    out = np.zeros((len(rows), V), np.float64)
+    rc = lib().oracle_lm_head_logits(_p(hidden), _p(w), _p(rows), len(rows), H, V, _p(out))
+    if rc:
+        raise ValueError("oracle_lm_head_logits rc=%d" % rc)
+    return out
+
+
+def argmax_rows_f64(x):
+    """First maximum of each row of a float64 array."""
+    x = _c(x, np.float64)
+    V = x.shape[-1]
+    out = np.zeros((x.size // V,), np.int32)
+    lib().oracle_argmax_rows_f64(_p(x), x.size // V, V, _p(out))
+    return out.reshape(x.shape[:-1])

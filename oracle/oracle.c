@@ -297,6 +297,44 @@ int oracle_argmax_rows(const float* logits, int64_t rows, int V, int32_t* out) {
   return 0;
 }
 
+/* ---------------------------------------------------------------------------
+ * Teacher logits from the final hidden states.
+ * [EP] 2.C: the teacher evaluates every speculative token in one batched pass;
+ * its greedy choice at node u is the argmax over the vocabulary of the LM-head
+ * logits, logit[u][v] = sum_h hidden[u][h] * W[v][h] (W: [V][H], bf16 inputs).
+ * The sum is taken in double precision: every bf16 product is exact in double,
+ * so the only rounding is that of the double accumulation.
+ * rows: nsel row indices into hidden [R][H]; out [nsel][V] double.
+ * ------------------------------------------------------------------------- */
+int oracle_lm_head_logits(const uint16_t* hidden, const uint16_t* w, const int32_t* rows, int64_t nsel, int H,
+                          int V, double* out) {
+  if (H <= 0 || V <= 0) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < nsel; ++i) {
+    const uint16_t* x = hidden + (int64_t)rows[i] * H;
+    double* o = out + i * V;
+    for (int v = 0; v < V; ++v) {
+      const uint16_t* wr = w + (int64_t)v * H;
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h) acc += bf16_to_double(x[h]) * bf16_to_double(wr[h]);
+      o[v] = acc;
+    }
+  }
+  return 0;
+}
+
+/* First maximum of each double row (strict '>'), as for the fp32 logits. */
+int oracle_argmax_rows_f64(const double* x, int64_t rows, int V, int32_t* out) {
+  for (int64_t r = 0; r < rows; ++r) {
+    const double* a = x + r * V;
+    int best = 0;
+    for (int j = 1; j < V; ++j)
+      if (a[j] > a[best]) best = j;
+    out[r] = best;
+  }
+  return 0;
+}
+
 /* Brute force: every root-to-leaf path, its longest accepted prefix. */
 static void brute_force_best(const int32_t* par, const int32_t* draft, const int32_t* am, int M,
                              int* best_len, int* best_end) {
