@@ -1127,7 +1127,7 @@ def run_ours(args, cfg, world, rank, local):
     if rank != 0:
         return
     steps = args.steps
-    rec.pop("_kv_len", None)
+    kv_len0 = rec.pop("_kv_len")
     for r in per_config.values():
         r.pop("_kv_len", None)
     steps = rec.get("steps_timed", args.steps)
@@ -1135,8 +1135,7 @@ def run_ours(args, cfg, world, rank, local):
         "metric": METRIC, "value": rec["nodes_per_s"], "unit": "nodes/s", "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_dict(dataclasses.replace(cfg, rounds=rec.get("rounds", cfg.rounds)), world,
-                              rec["_kv_len"]),
+        "config": config_dict(dataclasses.replace(cfg, rounds=rec.get("rounds", cfg.rounds)), world, kv_len0),
         "timing": GPU_TIMING,
         "layers_physical": rec["layers_physical"], "step_scaling": rec["step_scaling"],
         "ms_per_step_measured": rec.get("ms_per_step_measured", rec["ms_per_step"]),

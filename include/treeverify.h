@@ -225,6 +225,34 @@ tv_status tree_accept(const float* logits, const int32_t* draft, const int32_t* 
                       int32_t* bonus, tv_stream_t stream);
 
 /*
+ * tree_accept_lm_head -- tree_accept with the teacher's LM head fused in: the
+ * logits logit[b][u][v] = sum_h hidden[b][u][h] * w_lm[v][h] are formed tile by
+ * tile on the tensor cores and reduced to their first maximum on the spot, so
+ * the [B][M+1][V] logits are never written; the acceptance walk then runs as in
+ * tree_accept.  [EAGLE-Pangu, methodology C: one batched teacher pass over all
+ * speculative tokens, whose greedy choice at each node is the argmax of its
+ * logits; results: accepted length per verification step.]
+ *
+ *   hidden     bf16 [B][M+1][H]   in (final hidden state of every tree node),
+ *              16-byte aligned
+ *   w_lm       bf16 [V][H]        in (LM-head weights), 16-byte aligned
+ *   draft, parent, depth, anc_mask, status, argmax, accept_len, path, bonus:
+ *              as for tree_accept (argmax = first index of the row maximum of
+ *              the fp32-accumulated logits)
+ *   workspace  device scratch of tree_accept_lm_head_workspace_size(B, M) bytes,
+ *              8-byte aligned; no initialisation needed, dead after the call
+ *   H a multiple of 64; V >= 1.
+ * A tile whose pipeline wait gave up marks its rows' sequences TV_SEQ_TIMEOUT.
+ */
+size_t tree_accept_lm_head_workspace_size(int B, int M);
+
+tv_status tree_accept_lm_head(const uint16_t* hidden, const uint16_t* w_lm, const int32_t* draft,
+                              const int32_t* parent, const int32_t* depth, const uint32_t* anc_mask,
+                              int32_t* status, int B, int M, int H, int V, int max_depth, int32_t* argmax,
+                              int32_t* accept_len, int32_t* path, int32_t* bonus, void* workspace,
+                              size_t workspace_bytes, tv_stream_t stream);
+
+/*
  * kv_commit_realign -- commit the accepted path into the KV cache of every
  * layer and, in left-padded mode, repad the batch.  [EAGLE-Pangu, methodology A:
  * path-index commit; Batch Speculative Decoding Done Right, methodology:

@@ -23,6 +23,8 @@ from ._lib import (  # noqa: F401
     load,
     set_wait_limit_ns,
     tree_accept,
+    tree_accept_lm_head,
+    lm_head_workspace,
     tree_attention,
     tree_attention_workspace_size,
     tree_build_mask,

@@ -31,6 +31,8 @@ EXPORTS = (
     "tree_attention_noalloc_max_scratch",
     "tree_attention_noalloc",
     "tree_accept",
+    "tree_accept_lm_head_workspace_size",
+    "tree_accept_lm_head",
     "kv_commit_realign",
     "tree_kv_write",
     "tv_status_string",
@@ -66,9 +68,14 @@ def load(path: str = LIB_PATH):
     lib.tree_attention_noalloc.argtypes = [P, P, P, i64, P, P, P, P, i32, i32, i32, i32, i32, f32, P, P]
     lib.tree_attention_noalloc.restype = ctypes.c_int
     lib.tree_accept.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, P, P, P, P, P]
+    lib.tree_accept_lm_head_workspace_size.argtypes = [i32, i32]
+    lib.tree_accept_lm_head_workspace_size.restype = ctypes.c_size_t
+    lib.tree_accept_lm_head.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, ctypes.c_size_t,
+                                        P]
     lib.kv_commit_realign.argtypes = [P, P, i32, i32, i32, i32, i64, i32, P, P, P, i32, P, P, P, i32, P, P, P, i32, P]
     lib.tree_kv_write.argtypes = [P, P, P, P, i32, i32, i32, i32, i64, i32, P, P, P, f32, P, i32, P]
-    for name in ("tree_build_mask", "tree_attention", "tree_accept", "kv_commit_realign", "tree_kv_write"):
+    for name in ("tree_build_mask", "tree_attention", "tree_accept", "tree_accept_lm_head", "kv_commit_realign",
+                 "tree_kv_write"):
         getattr(lib, name).restype = ctypes.c_int
     lib.tv_status_string.argtypes = [ctypes.c_int]
     lib.tv_status_string.restype = ctypes.c_char_p
@@ -187,6 +194,34 @@ def tree_accept(logits, draft, parent, depth, anc_mask, status, max_depth, argma
                             B, n - 1, V, int(max_depth), _ptr(argmax), _ptr(accept_len), _ptr(path), _ptr(bonus),
                             _stream(stream))
     _check(rc, "tree_accept")
+
+
+def lm_head_workspace(B, M, device) -> torch.Tensor:
+    """A device buffer of tree_accept_lm_head_workspace_size bytes."""
+    nbytes = int(load().tree_accept_lm_head_workspace_size(B, M))
+    return torch.empty((max(nbytes, 8) + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+
+def tree_accept_lm_head(hidden, w_lm, draft, parent, depth, anc_mask, status, max_depth, argmax, accept_len, path,
+                        bonus, workspace, stream=None):
+    """hidden bf16 [B][M+1][H], w_lm bf16 [V][H] -> argmax of hidden @ w_lm^T per node
+    (the logits are never stored), then the acceptance walk (as tree_accept)."""
+    B, n, H = hidden.shape
+    V = w_lm.shape[0]
+    _need(hidden, torch.bfloat16, (B, n, H), "hidden")
+    _need(w_lm, torch.bfloat16, (V, H), "w_lm")
+    for t, name in ((draft, "draft"), (parent, "parent"), (depth, "depth"), (argmax, "argmax")):
+        _need(t, torch.int32, (B, n), name)
+    _need(anc_mask, torch.int32, (B, n, (n + 31) // 32), "anc_mask")
+    _need(status, torch.int32, (B,), "status")
+    _need(accept_len, torch.int32, (B,), "accept_len")
+    _need(path, torch.int32, (B, int(max_depth) + 1), "path")
+    _need(bonus, torch.int32, (B,), "bonus")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = load().tree_accept_lm_head(_ptr(hidden), _ptr(w_lm), _ptr(draft), _ptr(parent), _ptr(depth), _ptr(anc_mask),
+                                    _ptr(status), B, n - 1, H, V, int(max_depth), _ptr(argmax), _ptr(accept_len),
+                                    _ptr(path), _ptr(bonus), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "tree_accept_lm_head")
 
 
 def kv_commit_realign(k_layer_ptrs, v_layer_ptrs, B, Hkv, D, S_cap, M, path, accept_len, status, max_depth,

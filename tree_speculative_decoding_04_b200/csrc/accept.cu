@@ -205,6 +205,15 @@ __global__ void __launch_bounds__(kMaxRows) accept_walk_kernel(
 }
 
 }  // namespace
+
+tv_status launch_accept_walk(const int32_t* argmax, const int32_t* draft, const int32_t* parent,
+                             const int32_t* depth, const uint32_t* anc_mask, int32_t* status, int B, int M,
+                             int max_depth, int32_t* accept_len, int32_t* path, int32_t* bonus, cudaStream_t s) {
+  const int threads = 32 * ((M + 1 + 31) / 32);
+  return launch(accept_walk_kernel, dim3(B), dim3(threads), 0, s, 1, true, argmax, draft, parent, depth, anc_mask,
+                status, M, max_depth, accept_len, path, bonus);
+}
+
 }  // namespace tv
 
 extern "C" tv_status tree_accept(const float* logits, const int32_t* draft, const int32_t* parent,
@@ -234,7 +243,6 @@ extern "C" tv_status tree_accept(const float* logits, const int32_t* draft, cons
   tv_status r = launch(accept_argmax_kernel, dim3((unsigned)(rows * nsplit)), dim3(kArgmaxThreads), 0, s, nsplit,
                        true, logits, V, chunk, nsplit, argmax);
   if (r != TV_OK) return r;
-  const int threads = 32 * ((M + 1 + 31) / 32);
-  return launch(accept_walk_kernel, dim3(B), dim3(threads), 0, s, 1, true, (const int32_t*)argmax, draft, parent,
-                depth, anc_mask, status, M, max_depth, accept_len, path, bonus);
+  return launch_accept_walk(argmax, draft, parent, depth, anc_mask, status, B, M, max_depth, accept_len, path,
+                            bonus, s);
 }

@@ -106,6 +106,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -207,6 +214,13 @@ tv_status record_cuda_error(cudaError_t e);
 // Limit (ns) of the pipeline waits of the next attention launches
 // (tv_set_wait_limit_ns); kWaitLimitNs unless a test shortened it.
 uint64_t pipeline_wait_limit_ns();
+
+// The acceptance walk of tree_accept (accept.cu) on a per-node argmax that is
+// already in device memory: accepted = ancestors all matched, endpoint =
+// deepest accepted node (lowest row on ties), path / accept_len / bonus.
+tv_status launch_accept_walk(const int32_t* argmax, const int32_t* draft, const int32_t* parent,
+                             const int32_t* depth, const uint32_t* anc_mask, int32_t* status, int B, int M,
+                             int max_depth, int32_t* accept_len, int32_t* path, int32_t* bonus, cudaStream_t s);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
