@@ -75,6 +75,9 @@ def parse(argv=None):
     ap.add_argument("--rounds", type=int, default=0, help="rounds of a multi-round workload (0: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--profile", choices=["attention", "lm_head", "commit"], default=None,
+                    help="profiling run: a few launches of one kernel on one layer of the workload, no timing")
+    ap.add_argument("--batch", type=int, default=0, help="profiling run: sequences (0: the workload's)")
     return ap.parse_args(argv)
 
 
@@ -1153,9 +1156,69 @@ def run_ours(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args, cfg):
+    """A few launches of one kernel on one layer of the workload (optionally
+    fewer sequences), for an ncu capture: small enough to capture, inputs still
+    larger than L2 for the DRAM counters.  Prints the launch's algorithmic
+    bytes and flops so that the captured counters can be set against them."""
+    import tree_speculative_decoding_04_b200 as tv
+
+    device = torch.device("cuda", 0)
+    if args.batch:
+        cfg = dataclasses.replace(cfg, B=args.batch)
+    cfg = dataclasses.replace(cfg, L=1)
+    stream = torch.cuda.current_stream(device)
+    if args.profile == "lm_head":
+        H = cfg.Hq * cfg.D
+        g = W.torch_generator(args.seed, device)
+        rng = np.random.default_rng(args.seed)
+        parent = W.make_parents(cfg, rng)
+        n = cfg.M + 1
+        hidden = W.randn_bf16((cfg.B, n, H), g, device)
+        w = W.randn_bf16((cfg.V, H), g, device, sigma=H ** -0.5)
+        par = torch.as_tensor(parent, device=device)
+        anc = torch.zeros((cfg.B, n, (n + 31) // 32), dtype=torch.int32, device=device)
+        depth = torch.zeros((cfg.B, n), dtype=torch.int32, device=device)
+        status = torch.zeros((cfg.B,), dtype=torch.int32, device=device)
+        tv.tree_build_mask(par, cfg.max_depth, anc, depth, status)
+        draft = torch.zeros((cfg.B, n), dtype=torch.int32, device=device)
+        am = torch.zeros((cfg.B, n), dtype=torch.int32, device=device)
+        al = torch.zeros((cfg.B,), dtype=torch.int32, device=device)
+        path = torch.zeros((cfg.B, cfg.max_depth + 1), dtype=torch.int32, device=device)
+        bonus = torch.zeros((cfg.B,), dtype=torch.int32, device=device)
+        ws = tv.lm_head_workspace(cfg.B, cfg.M, device)
+        for _ in range(3):
+            tv.tree_accept_lm_head(hidden, w, draft, par, depth, anc, status, cfg.max_depth, am, al, path, bonus, ws)
+        torch.cuda.synchronize()
+        rows = cfg.B * n
+        print(json.dumps({"profile": "lm_head", "workload": cfg.name, "B": cfg.B, "rows": rows, "H": H, "V": cfg.V,
+                          "flops_per_launch": 2 * rows * H * cfg.V,
+                          "bytes_per_launch": cfg.V * H * 2 + rows * H * 2}))
+        return
+    ver, host = build_workload(cfg, args.seed, device)
+    with torch.cuda.stream(stream):
+        ver.build_mask(stream)
+        for _ in range(3):
+            if args.profile == "attention":
+                ver.attention(0, stream, prefix_ready=True)
+            else:
+                ver.kv_start.copy_(torch.as_tensor(host["kv_start"], device=device))
+                ver.kv_len.copy_(torch.as_tensor(host["kv_len"], device=device))
+                ver.accept(stream)
+                ver.commit(stream)
+    torch.cuda.synchronize()
+    depth = ver.depth.cpu().numpy()
+    print(json.dumps({"profile": args.profile, "workload": cfg.name, "B": cfg.B,
+                      "attention_bytes_per_launch": attention_bytes(cfg, host["kv_len"]),
+                      "attention_flops_per_launch": attention_flops(cfg, host["kv_len"], depth)}))
+
+
 def main(argv=None):
     ap_args = parse(argv)
     cfg = W.CONFIGS[ap_args.config]
+    if ap_args.profile:
+        run_profile(ap_args, cfg)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -4,10 +4,11 @@ and into tree_attention's query staging (TV_ATTN_ROPE), against the oracle.
 Tree positions: node u of sequence b sits at kv_len[b] + depth[b][u] (position-ID
 contiguity, "Batch Speculative Decoding Done Right", section 2).  The kernels
 form each angle in double precision and rotate in single precision; the oracle
-works in double throughout and rounds once to bf16.  K rows are therefore
-compared to within one bf16 unit in the last place (with nearly all equal), V
-rows and every cell outside the tree rows bit for bit, attention at the usual
-tolerance.
+works in double throughout and rounds once to bf16.  V rows and every cell
+outside the tree rows are compared bit for bit, attention at the usual
+tolerance.  K rows: within half a bf16 unit of a value within the fp32 error
+of the exact rotation (absolute near zero, where x cos - y sin cancels), and
+nearly all equal to the oracle's own rounding.
 """
 import numpy as np
 import pytest
@@ -23,10 +24,8 @@ pytestmark = pytest.mark.gpu
 THETA = 10000.0
 
 
-def _ordered(u16):
-    """bf16 bit patterns -> integers in the order of the values they encode."""
-    x = np.asarray(u16, np.uint16).astype(np.int32)
-    return np.where(x >= 0x8000, 0x8000 - x, x)
+def _bits_to_f64(u16):
+    return (np.asarray(u16, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def _tree_rows(st, cfg):
@@ -52,14 +51,30 @@ def test_kv_write_rotates_k_rows(orc, name):
                       depth=depth.cpu().numpy(), rope_base=THETA)
     gk, gv = W.bf16_bits(st.k), W.bf16_bits(st.v)
     np.testing.assert_array_equal(gv, vh[0])  # V rows copied, nothing else touched
-    diff = np.abs(_ordered(gk) - _ordered(kh[0]))
-    assert diff.max() <= 1, f"K rows differ by {diff.max()} bf16 ulps"
-    assert (diff != 0).mean() < 1e-3, f"{(diff != 0).mean():.2e} of the K elements differ by one ulp"
     mask = np.ones(gk.shape[:3], bool)
     for b in range(cfg.B):
         c0 = int(st.kv_start[b] + st.kv_len[b])
         mask[b, :, c0:c0 + cfg.M + 1] = False
     np.testing.assert_array_equal(gk[mask], k0[mask])  # outside the tree rows: untouched
+    # the rotated rows: within rounding of a value within the fp32 error of the
+    # exact rotation (x cos - y sin cancels, so near zero the bound is absolute,
+    # scaled by |x| + |y|), and nearly all equal to the oracle's own rounding
+    n, D = cfg.M + 1, cfg.D
+    raw = _bits_to_f64(W.bf16_bits(tk)[0])  # [B][Hkv][n][D]
+    dep = depth.cpu().numpy()
+    gpu_rows = np.stack([gk[b, :, int(st.kv_start[b] + st.kv_len[b]):int(st.kv_start[b] + st.kv_len[b]) + n]
+                         for b in range(cfg.B)])
+    for b in range(cfg.B):
+        pos = (int(st.kv_len[b]) + dep[b]).astype(np.float64)
+        for h in range(cfg.Hkv):
+            exact = orc.rope_rows(raw[b, h], pos, THETA)
+            mag = np.abs(raw[b, h]) + np.abs(np.roll(raw[b, h], D // 2, axis=1))
+            err = np.abs(_bits_to_f64(gpu_rows[b, h]) - exact)
+            bound = 2.0 ** -8 * np.abs(exact) + 2.0 ** -20 * mag
+            assert (err <= bound).all(), f"K row rotation off by {float((err - bound).max()):.3e} (b={b}, h={h})"
+    mismatch = (gpu_rows != np.stack([kh[0][b, :, int(st.kv_start[b] + st.kv_len[b]):
+                                              int(st.kv_start[b] + st.kv_len[b]) + n] for b in range(cfg.B)]))
+    assert mismatch.mean() < 1e-2, f"{mismatch.mean():.2e} of the K elements differ from the oracle's rounding"
 
 
 @pytest.mark.parametrize("name,sampled", [("tiny", False), ("mha7b", False), ("eqspec", False),

@@ -41,7 +41,7 @@ namespace {
 constexpr int kTcThreads = 192;
 constexpr int kRows = 128;
 constexpr int kTmemCols = 256;
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 8;
 constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
 constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
 constexpr float kRescaleThreshold = 8.0f;        // log2 domain
@@ -645,6 +645,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
 #ifndef TV_TC_ONE_PER_SM
 #define TV_TC_ONE_PER_SM 1
 #endif
+// ring depths (K, V) of a CTA that has its SM to itself
+#ifndef TV_TC_K_RING_SOLO
+#define TV_TC_K_RING_SOLO 3
+#endif
+#ifndef TV_TC_V_RING_SOLO
+#define TV_TC_V_RING_SOLO 6
+#endif
 
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& lp) {
   int dev = 0, sms = 148;
@@ -670,8 +677,8 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   const bool two_per_sm = !TV_TC_ONE_PER_SM || ctas > sms;
   // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
   // one CTA per SM: K ring 3, V ring up to 6
-  lp.stages = two_per_sm ? 2 : std::min(3, std::max(2, lp.tiles_per_split));
-  lp.v_stages = two_per_sm ? 3 : std::min(kMaxStages, std::max(2, lp.tiles_per_split));
+  lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
+  lp.v_stages = two_per_sm ? 3 : std::min(TV_TC_V_RING_SOLO, std::max(2, lp.tiles_per_split));
   const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
   lp.smem = std::max(smem_min, kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem));
   lp.ws_bytes = lp.nsplit > 1 ? (size_t)units * lp.nsplit * kRows * (128 + 2) * sizeof(float) : 0;
