@@ -29,65 +29,39 @@ namespace {
 constexpr int kWriteThreads = 256;
 constexpr int kWriteUnroll = 4;
 
-// Rotary variant of the K rows: one work item per pair of 16-byte chunks (c,
-// c + RV/2) of a K row, rotated to position kv_len + depth[b][r].
-__global__ void __launch_bounds__(kWriteThreads) kv_write_rope_k_kernel(
-    uint16_t* const* __restrict__ k_layers, const uint4* __restrict__ tree_k, int B, int Hkv, int RV,
-    int64_t S_cap, int M, const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len,
-    const int32_t* __restrict__ depth, const int32_t* __restrict__ slot, int n_slots, int64_t items,
-    const __grid_constant__ RopeFreqs fr) {
-  pdl_wait_primary();
-  pdl_launch_dependents();
-  const int n = M + 1;
-  const int half = RV / 2;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < items; w += stride) {
-    const int c = (int)(w % half);
-    const int64_t row = w / half;  // ((l * B + b) * Hkv + h) * n + r
-    const int r = (int)(row % n);
-    const int64_t run = row / n;
-    const int h = (int)(run % Hkv);
-    const int64_t lb = run / Hkv;
-    const int b = (int)(lb % B);
-    const int l = (int)(lb / B);
-    const int sl = cache_slot(slot, b, n_slots);
-    if (sl < 0) continue;
-    const int32_t ks = kv_start[sl], kl = kv_len[sl];
-    if (!geometry_ok(ks, kl, M, S_cap)) continue;
-    uint4 lo = tree_k[row * RV + c], hi = tree_k[row * RV + c + half];
-    rope_rotate8(lo, hi, kl + depth[(int64_t)b * n + r], fr.f, 8 * c);
-    uint4* cache = reinterpret_cast<uint4*>(k_layers[l]) + (((int64_t)sl * Hkv + h) * S_cap + ks + kl + r) * RV;
-    cache[c] = lo;
-    cache[c + half] = hi;
-  }
-}
-
-// kv = 0: K and V rows (plain copy); kv = 1 only V rows (the K rows are
-// written by the rotary kernel).
+// One launch for the whole append.  Work items: without rotation, 16-byte
+// units of K then V; with rotation, the K rows as pairs of 16-byte chunks (c,
+// c + RV/2) rotated to position kv_len + depth[b][r], then the V units.
 __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
     uint16_t* const* __restrict__ k_layers, uint16_t* const* __restrict__ v_layers,
     const uint4* __restrict__ tree_k, const uint4* __restrict__ tree_v, int B, int Hkv, int RV, int64_t S_cap,
     int M, const int32_t* __restrict__ kv_start, const int32_t* __restrict__ kv_len,
-    const int32_t* __restrict__ slot, int n_slots, int64_t per_kv, int v_only) {
+    const int32_t* __restrict__ slot, int n_slots, int64_t per_kv, const int32_t* __restrict__ depth,
+    const __grid_constant__ RopeFreqs fr) {
   pdl_wait_primary();
   pdl_launch_dependents();
   const int n = M + 1;
-  const int64_t first = v_only ? per_kv : 0;
-  const int64_t total = 2 * per_kv - first;  // 16-byte units: K then V
+  const bool rope = depth != nullptr;
+  const int half = RV / 2;
+  const int64_t k_items = rope ? per_kv / 2 : per_kv;  // K work items
+  const int64_t total = k_items + per_kv;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < total;
        base += stride * kWriteUnroll) {
-    uint4 val[kWriteUnroll];
+    uint4 val[kWriteUnroll], val2[kWriteUnroll];
     uint4* dst[kWriteUnroll];
+    int dst2_off[kWriteUnroll];  // second chunk of a rotated pair (0: none)
 #pragma unroll
     for (int t = 0; t < kWriteUnroll; ++t) {
       dst[t] = nullptr;
-      const int64_t u = first + base + (int64_t)t * stride;
-      if (u >= 2 * per_kv) continue;
-      const int kv = u >= per_kv;
-      const int64_t w = kv ? u - per_kv : u;  // index inside [L][B][Hkv][n][RV]
-      const int c = (int)(w % RV);
-      const int64_t row = w / RV;  // ((l * B + b) * Hkv + h) * n + r
+      dst2_off[t] = 0;
+      const int64_t u = base + (int64_t)t * stride;
+      if (u >= total) continue;
+      const bool is_k = u < k_items;
+      const int units = (is_k && rope) ? half : RV;  // items per row
+      const int64_t w = is_k ? u : u - k_items;
+      const int c = (int)(w % units);
+      const int64_t row = w / units;  // ((l * B + b) * Hkv + h) * n + r
       const int r = (int)(row % n);
       const int64_t run = row / n;
       const int h = (int)(run % Hkv);
@@ -98,13 +72,24 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(
       if (sl < 0) continue;
       const int32_t ks = kv_start[sl], kl = kv_len[sl];
       if (!geometry_ok(ks, kl, M, S_cap)) continue;
-      val[t] = kv ? tree_v[w] : tree_k[w];
-      uint4* cache = reinterpret_cast<uint4*>((kv ? v_layers : k_layers)[l]);
-      dst[t] = cache + (((int64_t)sl * Hkv + h) * S_cap + ks + kl + r) * RV + c;
+      uint4* cache = reinterpret_cast<uint4*>((is_k ? k_layers : v_layers)[l]) +
+                     (((int64_t)sl * Hkv + h) * S_cap + ks + kl + r) * RV;
+      if (is_k && rope) {
+        val[t] = tree_k[row * RV + c];
+        val2[t] = tree_k[row * RV + c + half];
+        rope_rotate8(val[t], val2[t], kl + depth[(int64_t)b * n + r], fr.f, 8 * c);
+        dst2_off[t] = half;
+      } else {
+        val[t] = is_k ? tree_k[row * RV + c] : tree_v[row * RV + c];
+      }
+      dst[t] = cache + c;
     }
 #pragma unroll
     for (int t = 0; t < kWriteUnroll; ++t)
-      if (dst[t]) *dst[t] = val[t];
+      if (dst[t]) {
+        *dst[t] = val[t];
+        if (dst2_off[t]) dst[t][dst2_off[t]] = val2[t];
+      }
   }
 }
 
@@ -132,21 +117,12 @@ extern "C" tv_status tree_kv_write(uint16_t* const* k_layers, uint16_t* const* v
   if (e != cudaSuccess) return record_cuda_error(e);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (rope) {
-    RopeFreqs fr;
-    rope_freqs((double)rope_theta, D, fr);
-    const int64_t items = per_kv / 2;
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((items + kWriteThreads - 1) / kWriteThreads,
-                                                                  (int64_t)sms * 8));
-    tv_status r = launch(kv_write_rope_k_kernel, dim3((unsigned)blocks), dim3(kWriteThreads), 0, s, 1, true,
-                         k_layers, reinterpret_cast<const uint4*>(tree_k), B, Hkv, D / 8, S_cap, M, kv_start, kv_len,
-                         depth, slot, slot ? n_slots : B, items, fr);
-    if (r != TV_OK) return r;
-  }
-  const int64_t units = rope ? per_kv : 2 * per_kv;
+  RopeFreqs fr;
+  rope_freqs(rope ? (double)rope_theta : 2.0, D, fr);
+  const int64_t units = (rope ? per_kv / 2 : per_kv) + per_kv;
   const int64_t need = (units + (int64_t)kWriteThreads * kWriteUnroll - 1) / ((int64_t)kWriteThreads * kWriteUnroll);
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(need, (int64_t)sms * 8));
   return launch(kv_write_kernel, dim3((unsigned)blocks), dim3(kWriteThreads), 0, s, 1, true, k_layers, v_layers,
                 reinterpret_cast<const uint4*>(tree_k), reinterpret_cast<const uint4*>(tree_v), B, Hkv, D / 8, S_cap,
-                M, kv_start, kv_len, slot, slot ? n_slots : B, per_kv, rope ? 1 : 0);
+                M, kv_start, kv_len, slot, slot ? n_slots : B, per_kv, rope ? depth : (const int32_t*)nullptr, fr);
 }

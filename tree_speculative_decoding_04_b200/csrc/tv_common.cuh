@@ -177,14 +177,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------- rotary embedding
 // cos and sin of the angle pos * inv_freq.  The angle is formed and reduced to
 // [-pi, pi] in double precision (two-part 2 pi, Cody-Waite style), so that the
-// single-precision sine and cosine see an argument accurate to float rounding
-// even at positions of tens of thousands.
+// hardware sine and cosine (MUFU, absolute error below 4e-7 on [-pi, pi]) see
+// an argument accurate to float rounding even at positions of tens of
+// thousands.
 __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
   const double a = (double)pos * inv_freq;
   const double k = rint(a * 0.15915494309189535);   // a / (2 pi), nearest integer
   double r = fma(-k, 6.283185307179586, a);         // 2 pi, leading double
   r = fma(-k, 2.4492935982947064e-16, r);           // 2 pi, remainder
-  sincosf((float)r, &s, &c);
+  const float rf = (float)r;
+  s = __sinf(rf);
+  c = __cosf(rf);
 }
 
 // Rotate 8 pairs: lo holds elements i0 .. i0+7 of a row, hi the elements
