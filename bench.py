@@ -842,6 +842,78 @@ def measure_rounds(args, cfg, world, device, rounds, replays, warmup, with_clock
     return rec, dict(ver=ver, host=host, clk=clk, stream=stream)
 
 
+def measure_lm_head(args, cfg, device, reps=5):
+    """tree_accept_lm_head on the workload's tree rows: hidden states [B][M+1][H]
+    (H = Hq * D) against synthetic LM-head weights [V][H], the argmax fused into
+    the GEMM's epilogue, then the acceptance walk.  Beside it, the unfused path
+    it replaces: the logits written by a cuBLAS bf16 GEMM (through torch),
+    widened to fp32, then tree_accept."""
+    import tree_speculative_decoding_04_b200 as tv
+
+    H = cfg.Hq * cfg.D
+    n = cfg.M + 1
+    rng = np.random.default_rng(args.seed + 3)
+    g = W.torch_generator(args.seed + 3, device)
+    parent = W.make_parents(cfg, rng)
+    hidden = W.randn_bf16((cfg.B, n, H), g, device)
+    w = W.randn_bf16((cfg.V, H), g, device, sigma=H ** -0.5)
+    rows = cfg.B * n
+    i32 = dict(dtype=torch.int32, device=device)
+    par = torch.as_tensor(parent, device=device)
+    anc = torch.zeros((cfg.B, n, (n + 31) // 32), **i32)
+    depth = torch.zeros((cfg.B, n), **i32)
+    status = torch.zeros((cfg.B,), **i32)
+    tv.tree_build_mask(par, cfg.max_depth, anc, depth, status)
+    logits = torch.matmul(hidden.reshape(rows, H), w.T).float().reshape(cfg.B, n, cfg.V)
+    draft = torch.as_tensor(W.plant_drafts(logits, parent, cfg.p_plant, rng), device=device)
+    am = torch.zeros((cfg.B, n), **i32)
+    al = torch.zeros((cfg.B,), **i32)
+    path = torch.zeros((cfg.B, cfg.max_depth + 1), **i32)
+    bonus = torch.zeros((cfg.B,), **i32)
+    ws = tv.lm_head_workspace(cfg.B, cfg.M, device)
+    stream = torch.cuda.Stream(device)
+
+    def fused():
+        tv.tree_accept_lm_head(hidden, w, draft, par, depth, anc, status, cfg.max_depth, am, al, path, bonus, ws,
+                               stream)
+
+    def unfused():
+        lg = torch.matmul(hidden.reshape(rows, H), w.T).float().reshape(cfg.B, n, cfg.V)
+        tv.tree_accept(lg, draft, par, depth, anc, status, cfg.max_depth, am, al, path, bonus, stream)
+
+    with torch.cuda.stream(stream):
+        fused()
+        unfused()
+    torch.cuda.synchronize()
+    g_f = capture(fused, stream)
+    with torch.cuda.stream(stream):
+        g_f.replay()
+    f_ms = event_time(g_f.replay, reps, stream)
+    del g_f
+    with torch.cuda.stream(stream):
+        u_ms = event_time(unfused, reps, stream)
+    same = None
+    with torch.cuda.stream(stream):
+        fused()
+    torch.cuda.synchronize()
+    a_f = am.clone()
+    with torch.cuda.stream(stream):
+        unfused()
+    torch.cuda.synchronize()
+    same = float((a_f == am).float().mean().item())
+    hbm, tflops, peak_kind = peaks()
+    flops = 2 * rows * H * cfg.V
+    nbytes = cfg.V * H * 2 + rows * H * 2
+    r = roofline_entry(nbytes, flops, f_ms, hbm, tflops, peak_kind, None, "lm_head_argmax_kernel")
+    del hidden, w, logits
+    torch.cuda.empty_cache()
+    return {"rows": rows, "H": H, "V": cfg.V, "fused_us": f_ms * 1e3, "unfused_us": u_ms * 1e3,
+            "speedup_vs_unfused": u_ms / f_ms, "argmax_agreement_with_unfused": same,
+            "logits_bytes_not_written": rows * cfg.V * 4, "roofline": r,
+            "note": "fused: tree_accept_lm_head (GEMM + argmax epilogue + walk); unfused: cuBLAS bf16 logits "
+                    "widened to fp32, then tree_accept"}
+
+
 def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
     """Cross-batch scheduling (EXSPEC) on the EQSPEC shapes: a pool of n_slots
     sequences whose prefix lengths come from a few length buckets (drawn from the
@@ -1114,6 +1186,12 @@ def run_ours(args, cfg, world, rank, local):
                 per_config[name] = r
             except Exception as e:  # a secondary workload must not void the headline line
                 per_config[name] = {"error": repr(e)[:300]}
+                torch.cuda.empty_cache()
+        for name in ("mha7b", "eqspec", "b32gqa", "stress"):
+            try:
+                per_config.setdefault(name, {})["lm_head"] = measure_lm_head(args, W.CONFIGS[name], device)
+            except Exception as e:
+                per_config.setdefault(name, {})["lm_head"] = {"error": repr(e)[:300]}
                 torch.cuda.empty_cache()
         try:
             per_config["exspec"] = measure_exspec(args, W.CONFIGS["eqspec"], device)

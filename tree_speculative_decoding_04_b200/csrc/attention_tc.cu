@@ -646,6 +646,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
 #define TV_TC_ONE_PER_SM 1
 #endif
 // ring depths (K, V) of a CTA that has its SM to itself
+//   TV_TC_FORCE_SOLO    1: one CTA per SM (deep rings) even for grids of
+//                       several waves
+#ifndef TV_TC_FORCE_SOLO
+#define TV_TC_FORCE_SOLO 0
+#endif
 #ifndef TV_TC_K_RING_SOLO
 #define TV_TC_K_RING_SOLO 3
 #endif
@@ -674,7 +679,7 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
   // never waits on a CTA that is itself waiting), else one CTA per SM.
   const int64_t ctas = units * lp.nsplit;
-  const bool two_per_sm = !TV_TC_ONE_PER_SM || ctas > sms;
+  const bool two_per_sm = !TV_TC_FORCE_SOLO && (!TV_TC_ONE_PER_SM || ctas > sms);
   // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
   // one CTA per SM: K ring 3, V ring up to 6
   lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
