@@ -35,6 +35,37 @@
 
 namespace cg = cooperative_groups;
 
+// Tuning (compile-time, so that a sweep can rebuild with -D):
+//   TV_TC_SPLIT_FACTOR  key splits are added while units * splits stays within
+//                       this many CTAs per SM
+//   TV_TC_ONE_PER_SM    1: a grid that fits one wave gets one CTA per SM with
+//                       deeper rings; 0: every CTA stays within half an SM's
+//                       shared memory, so the next launch's CTAs can become
+//                       resident beside it and start streaming early
+#ifndef TV_TC_SPLIT_FACTOR
+#define TV_TC_SPLIT_FACTOR 2
+#endif
+#ifndef TV_TC_ONE_PER_SM
+#define TV_TC_ONE_PER_SM 1
+#endif
+// ring depths (K, V) of a CTA that has its SM to itself
+//   TV_TC_POLY_EXP_PAIRS  of every 8 pairs of probabilities, how many are
+//                       exponentiated on the FMA pipe (the rest on the MUFU)
+#ifndef TV_TC_POLY_EXP_PAIRS
+#define TV_TC_POLY_EXP_PAIRS 0
+#endif
+//   TV_TC_FORCE_SOLO    1: one CTA per SM (deep rings) even for grids of
+//                       several waves
+#ifndef TV_TC_FORCE_SOLO
+#define TV_TC_FORCE_SOLO 0
+#endif
+#ifndef TV_TC_K_RING_SOLO
+#define TV_TC_K_RING_SOLO 3
+#endif
+#ifndef TV_TC_V_RING_SOLO
+#define TV_TC_V_RING_SOLO 6
+#endif
+
 namespace tv {
 namespace {
 
@@ -443,9 +474,16 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          float a0, a1;
-          f2_unpack(f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), sc2, nm2), a0, a1);
-          const float p0 = fast_exp2(a0), p1 = fast_exp2(a1);
+          const uint64_t arg = f2_fma(f2_pack(x[2 * j], x[2 * j + 1]), sc2, nm2);
+          float p0, p1;
+          if ((j & 7) < TV_TC_POLY_EXP_PAIRS) {  // a share of the pairs on the FMA pipe
+            f2_unpack(f2_exp2_poly(arg), p0, p1);
+          } else {
+            float a0, a1;
+            f2_unpack(arg, a0, a1);
+            p0 = fast_exp2(a0);
+            p1 = fast_exp2(a1);
+          }
           rs2[j & 3] = f2_add(rs2[j & 3], f2_pack(p0, p1));
           pk[j] = pack_bf16x2(p0, p1);
         }
@@ -631,32 +669,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
 }
 
 }  // namespace
-
-// Tuning of the launch plan (compile-time, so that a sweep can rebuild with -D):
-//   TV_TC_SPLIT_FACTOR  key splits are added while units * splits stays within
-//                       this many CTAs per SM
-//   TV_TC_ONE_PER_SM    1: a grid that fits one wave gets one CTA per SM with
-//                       deeper rings; 0: every CTA stays within half an SM's
-//                       shared memory, so the next launch's CTAs can become
-//                       resident beside it and start streaming early
-#ifndef TV_TC_SPLIT_FACTOR
-#define TV_TC_SPLIT_FACTOR 2
-#endif
-#ifndef TV_TC_ONE_PER_SM
-#define TV_TC_ONE_PER_SM 1
-#endif
-// ring depths (K, V) of a CTA that has its SM to itself
-//   TV_TC_FORCE_SOLO    1: one CTA per SM (deep rings) even for grids of
-//                       several waves
-#ifndef TV_TC_FORCE_SOLO
-#define TV_TC_FORCE_SOLO 0
-#endif
-#ifndef TV_TC_K_RING_SOLO
-#define TV_TC_K_RING_SOLO 3
-#endif
-#ifndef TV_TC_V_RING_SOLO
-#define TV_TC_V_RING_SOLO 6
-#endif
 
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& lp) {
   int dev = 0, sms = 148;

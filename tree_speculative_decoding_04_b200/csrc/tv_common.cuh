@@ -169,6 +169,31 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^a for a pair of floats on the FMA pipe instead of the MUFU: a = n + f with
+// n the nearest integer (the 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2];
+// 2^f by a cubic fitted to it (least squares at Chebyshev nodes, relative error
+// below 7.5e-5 -- far below the bf16 rounding of the probabilities), scaled by
+// 2^n through the exponent field.  Arguments below -125 are clamped there
+// (result about 2e-38, nothing that moves an fp32 sum of terms near 1).
+__device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t a) {
+  float a0, a1;
+  f2_unpack(a, a0, a1);
+  a = f2_pack(fmaxf(a0, -125.f), fmaxf(a1, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(a, magic);                                          // n in the low mantissa bits
+  const uint64_t fr = f2_fma(f2_add(t, f2_pack(-12582912.f, -12582912.f)), f2_pack(-1.f, -1.f), a);  // a - n
+  uint64_t p = f2_fma(f2_pack(0.055171613f, 0.055171613f), fr, f2_pack(0.24261113f, 0.24261113f));
+  p = f2_fma(p, fr, f2_pack(0.69326097f, 0.69326097f));
+  p = f2_fma(p, fr, f2_pack(0.99992806f, 0.99992806f));
+  float t0, t1, p0, p1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(p, p0, p1);
+  const int k = 0x4B400000;  // bits of 1.5 * 2^23
+  const float r0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - k) << 23));
+  const float r1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - k) << 23));
+  return f2_pack(r0, r1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
