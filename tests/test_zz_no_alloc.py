@@ -52,7 +52,8 @@ def _with_workspace(lib, cfg, st, anc, status, ks, kl, out, stream):
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=out.device)
     rc = lib.tree_attention(
         _p(st.q), _p(st.k), _p(st.v), st.S_cap, _p(ks), _p(kl), _p(anc), _p(status), cfg.B, cfg.M, cfg.Hq,
-        cfg.Hkv, cfg.D, ctypes.c_float(cfg.D ** -0.5), _p(out), _p(ws), nbytes, 0, ctypes.c_void_p(stream))
+        cfg.Hkv, cfg.D, ctypes.c_float(cfg.D ** -0.5), _p(out), _p(ws), nbytes, 0, None, ctypes.c_float(0.0), None, 0,
+        ctypes.c_void_p(stream))
     return rc, ws
 
 

@@ -480,8 +480,14 @@ tv_status prepare_attention(const uint16_t* q, const uint16_t* k, const uint16_t
   rope_freqs(rope ? (double)rope_theta : 2.0, D, p.rope);
   p.ws = nullptr;
   if ((int64_t)p.n_slots * Hkv > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
-  if (!encode_kv_map(&call.tmk, k, p.n_slots * Hkv, S_cap, D) || !encode_kv_map(&call.tmv, v, p.n_slots * Hkv, S_cap, D))
+  p.kv_4d = 0;
+  if (D == 128 && encode_kv_map_4d(&call.tmk, k, p.n_slots * Hkv, S_cap) &&
+      encode_kv_map_4d(&call.tmv, v, p.n_slots * Hkv, S_cap)) {
+    p.kv_4d = 1;
+  } else if (!encode_kv_map(&call.tmk, k, p.n_slots * Hkv, S_cap, D) ||
+             !encode_kv_map(&call.tmv, v, p.n_slots * Hkv, S_cap, D)) {
     return TV_ERR_INVALID_ARG;
+  }
   if (D == 128) return plan_attention_tc(B, M, Hq, Hkv, S_cap, call.plan);
   return TV_OK;
 }

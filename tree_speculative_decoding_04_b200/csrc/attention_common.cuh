@@ -30,6 +30,7 @@ struct AttnParams {
   const int32_t* depth; // [B][M+1] node depths (rotary positions kv_len + depth), TV_ATTN_ROPE only
   const int32_t* slot;  // [B] cache slot of each batch row, or null (slot = row)
   int n_slots;          // slots of the cache pool (B without a slot map)
+  int kv_4d;            // the K/V maps are 4-D (one 16 KB box per tile), else 3-D (two 8 KB boxes)
   RopeFreqs rope;       // inverse frequencies, TV_ATTN_ROPE only
   uint64_t wait_limit_ns;  // limit of the pipeline waits (the drain waits keep kWaitLimitNs)
   float* ws;            // split partials: [units][nsplit][128 rows][128] O, then [units][nsplit][128][2] (m, l)
@@ -50,6 +51,24 @@ inline EncodeTiledFn get_encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(f);
   });
   return fn;
+}
+
+// [B*Hkv][S_cap][128] bf16 as a 4-D tensor {64 columns, S_cap rows, 2 halves,
+// BH} (strides: row 256 B, half 128 B, head S_cap * 256 B) with boxes of 64 x 64
+// x 2 x 1: one 16 KB copy brings a whole 64-key tile, landing as [half][row][128
+// B] -- the layout of two 8 KB boxes -- with one copy instead of two.  Returns
+// false if the driver refuses the layout (the caller then uses the 3-D map).
+inline bool encode_kv_map_4d(CUtensorMap* map, const void* base, int BH, int64_t S_cap) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {64, (cuuint64_t)S_cap, 2, (cuuint64_t)BH};
+  cuuint64_t strides[3] = {256, 128, (cuuint64_t)S_cap * 256};
+  cuuint32_t box[4] = {64, (cuuint32_t)kKeyTile, 2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 // [B*Hkv][S_cap][D] bf16 -> boxes of 64 columns (128 B) x 64 rows, 128-byte swizzle.

@@ -173,19 +173,23 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     prefetch_tensormap(&tmv);
   }
   // zc_: the tensor-map row block of (cache slot, kv head)
+  // one 16 KB box per tile with the 4-D maps, else two 8 KB boxes
+  auto load_tile = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int zc_) {
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    if (p.kv_4d) {
+      tma_load_4d(dst, map, bar, 0, row, 0, zc_);
+    } else {
+      tma_load_3d(dst, map, bar, 0, row, zc_);
+      tma_load_3d(dst + kBoxBytes, map, bar, 64, row, zc_);
+    }
+  };
   auto issue_k = [&](int i, int32_t ks_, int k_lo_, int zc_) {
     const int s = i % k_stages;
-    uint8_t* dst = k_ring + s * kTileBytes;
-    mbar_arrive_expect_tx(&sh->k_full[s], kTileBytes);
-    tma_load_3d(dst, &tmk, &sh->k_full[s], 0, ks_ + k_lo_ + i * kKeyTile, zc_);
-    tma_load_3d(dst + kBoxBytes, &tmk, &sh->k_full[s], 64, ks_ + k_lo_ + i * kKeyTile, zc_);
+    load_tile(k_ring + s * kTileBytes, &tmk, &sh->k_full[s], ks_ + k_lo_ + i * kKeyTile, zc_);
   };
   auto issue_v = [&](int i, int32_t ks_, int k_lo_, int zc_) {
     const int s = i % v_stages;
-    uint8_t* dst = v_ring + s * kTileBytes;
-    mbar_arrive_expect_tx(&sh->v_full[s], kTileBytes);
-    tma_load_3d(dst, &tmv, &sh->v_full[s], 0, ks_ + k_lo_ + i * kKeyTile, zc_);
-    tma_load_3d(dst + kBoxBytes, &tmv, &sh->v_full[s], 64, ks_ + k_lo_ + i * kKeyTile, zc_);
+    load_tile(v_ring + s * kTileBytes, &tmv, &sh->v_full[s], ks_ + k_lo_ + i * kKeyTile, zc_);
   };
   // This sequence's key tiles are dealt evenly over the splits (ragged batches
   // would otherwise leave short sequences in one split).
@@ -244,10 +248,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         const int nt = min(kPrefetchTiles, nt_h);
         for (int i = 0; i < nt; ++i) {
           const int row = ks_h + k_lo_h + i * kKeyTile;
-          tma_prefetch_3d(&tmk, 0, row, sl_h * p.Hkv + hk);
-          tma_prefetch_3d(&tmk, 64, row, sl_h * p.Hkv + hk);
-          tma_prefetch_3d(&tmv, 0, row, sl_h * p.Hkv + hk);
-          tma_prefetch_3d(&tmv, 64, row, sl_h * p.Hkv + hk);
+          if (p.kv_4d) {
+            tma_prefetch_4d(&tmk, 0, row, 0, sl_h * p.Hkv + hk);
+            tma_prefetch_4d(&tmv, 0, row, 0, sl_h * p.Hkv + hk);
+          } else {
+            tma_prefetch_3d(&tmk, 0, row, sl_h * p.Hkv + hk);
+            tma_prefetch_3d(&tmk, 64, row, sl_h * p.Hkv + hk);
+            tma_prefetch_3d(&tmv, 0, row, sl_h * p.Hkv + hk);
+            tma_prefetch_3d(&tmv, 64, row, sl_h * p.Hkv + hk);
+          }
         }
       }
     }
