@@ -56,6 +56,10 @@ namespace cg = cooperative_groups;
 #endif
 //   TV_TC_FORCE_SOLO    1: one CTA per SM (deep rings) even for grids of
 //                       several waves
+//   TV_TC_PAIR          1: two query tiles per CTA when a unit has two or more
+#ifndef TV_TC_PAIR
+#define TV_TC_PAIR 1
+#endif
 #ifndef TV_TC_FORCE_SOLO
 #define TV_TC_FORCE_SOLO 0
 #endif
@@ -69,7 +73,6 @@ namespace cg = cooperative_groups;
 namespace tv {
 namespace {
 
-constexpr int kTcThreads = 192;
 constexpr int kRows = 128;
 constexpr int kTmemCols = 256;
 constexpr int kMaxStages = 8;
@@ -84,9 +87,9 @@ struct TcSmem {
   uint64_t k_empty[kMaxStages];
   uint64_t v_full[kMaxStages];
   uint64_t v_empty[kMaxStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_ready[2];  // PV_j completes a phase of o_ready[j % 2]
+  uint64_t s_full[2][2];   // [query pipe][S buffer]
+  uint64_t p_full[2][2];   // [query pipe][S buffer]
+  uint64_t o_ready[2][2];  // [query pipe][j % 2]: PV_j completes a phase
   uint64_t q_ready;
   uint64_t drain;
   uint32_t tmem_base;
@@ -107,44 +110,55 @@ __device__ __forceinline__ uint64_t anc_window(const uint32_t (&aw)[kMaxRows / 3
   return r;
 }
 
-// O += P_j V_j for key tile j (one thread), then release the K/V stage and
-// publish the new O.  Returns false if P_j never arrived.
-__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t t_s0, uint32_t t_o, int j,
-                                         int v_stages, uint64_t lim) {
+// O_q += P_{q,j} V_j for key tile j and every query pipe q < nq (one thread),
+// then release the V stage once every pipe has used it and publish each new
+// O.  Pipe q's TMEM block starts at column q * 256: S buffers at +0 / +64 (P_j
+// aliases S[j % 2]), O at +128.  Returns false if a P or V never arrived.
+__device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t tmem, int nq, int j, int v_stages,
+                                         uint64_t lim) {
   const uint32_t idesc_o = idesc_bf16(128, 128, 1);
   const int sb = j & 1, s = j % v_stages;
-  if (!mbar_wait(&sh->p_full[sb], (j >> 1) & 1, lim)) return false;
   if (!mbar_wait(&sh->v_full[s], (j / v_stages) & 1, lim)) return false;
-  tc_fence_after();
   const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
+  for (int q = 0; q < nq; ++q) {
+    if (!mbar_wait(&sh->p_full[q][sb], (j >> 1) & 1, lim)) return false;
+    tc_fence_after();
+    const uint32_t t_q = tmem + q * kTmemCols;
 #pragma unroll
-  for (int kk = 0; kk < kKeyTile / 16; ++kk)
-    mma_ts(t_o, t_s0 + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
-           (j > 0 || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < kKeyTile / 16; ++kk)
+      mma_ts(t_q + 128, t_q + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
+             (j > 0 || kk > 0) ? 1u : 0u);
+    tc_commit(&sh->o_ready[q][j & 1]);
+  }
   tc_commit(&sh->v_empty[s]);
-  tc_commit(&sh->o_ready[j & 1]);
   return true;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk,
-                                                                    const __grid_constant__ CUtensorMap tmv,
-                                                                    const __grid_constant__ AttnParams p) {
+// NQ query tiles per CTA share every K/V tile (NQ = 2: 8 softmax warps, all 512
+// TMEM columns, one CTA per SM); the query tiles of a (sequence, kv head) are
+// blockIdx.y * NQ + q.
+template <int NQ>
+__global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
+    tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                        const __grid_constant__ AttnParams p) {
   // The 128-byte-swizzled tiles need 1024-byte alignment.  The dynamic window
   // starts on such a boundary on this GPU; if it ever did not, every CTA treats
   // its sequence as failed (zero output, TV_SEQ_TIMEOUT) instead of computing.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const bool aligned_ok = (smem_u32(smem_raw) & 1023u) == 0;
-  uint8_t* q_s = smem;                              // [2][128][128 B]
+  uint8_t* q_s = smem;                              // [NQ][2][128][128 B]
   const int k_stages = p.stages, v_stages = p.v_stages;
-  uint8_t* k_ring = smem + kQBytes;                   // [k_stages][2 boxes of 64 rows x 128 B]
+  uint8_t* k_ring = smem + NQ * kQBytes;              // [k_stages][2 boxes of 64 rows x 128 B]
   uint8_t* v_ring = k_ring + k_stages * kTileBytes;   // [v_stages][2 boxes]
   TcSmem* sh = reinterpret_cast<TcSmem*>(v_ring + v_stages * kTileBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x;
-  const int qtile = blockIdx.y;
+  const int tiles_q = (p.rows_total + kRows - 1) / kRows;
+  const int qtile0 = blockIdx.y * NQ;                  // first query tile of this CTA
+  const int nq = min(NQ, tiles_q - qtile0);            // query tiles present (the last CTA may have fewer)
   const int bh = blockIdx.z;
   const int b = bh / p.Hkv;
   const int hk = bh - b * p.Hkv;
@@ -159,12 +173,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       mbar_init(&sh->v_full[s], 1);
       mbar_init(&sh->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sh->s_full[s], 1);
-      mbar_init(&sh->p_full[s], 4);
-    }
-    mbar_init(&sh->o_ready[0], 1);
-    mbar_init(&sh->o_ready[1], 1);
+    for (int q = 0; q < NQ; ++q)
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(&sh->s_full[q][s], 1);
+        mbar_init(&sh->p_full[q][s], 4);
+        mbar_init(&sh->o_ready[q][s], 1);
+      }
     mbar_init(&sh->drain, 1);
     fence_mbar_init();
   }
@@ -262,7 +276,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     }
   }
   if (warp >= 2) {
-    const int gr_h = qtile * kRows + (warp & 3) * 32 + lane;
+    const int gr_h = (qtile0 + ((warp - 2) >> 2)) * kRows + (warp & 3) * 32 + lane;
     if (gr_h < p.rows_total) {
       const uint16_t* qr = p.q + (((int64_t)b * (p.M + 1) + gr_h / p.G) * p.Hq + hk * p.G + gr_h % p.G) * 128;
       prefetch_l2(qr);
@@ -296,9 +310,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       if (i < k_stages && i >= npre_k) issue_k(i, ks, k_lo, zc);
       if (i < v_stages && i >= npre_v) issue_v(i, ks, k_lo, zc);
     }
+  const int pipe = warp >= 2 ? (warp - 2) >> 2 : 0;  // query pipe of a softmax warp
+  const int qtile = qtile0 + pipe;
+  uint8_t* q_pipe = q_s + pipe * kQBytes;
+  const uint32_t tq = (uint32_t)(pipe * kTmemCols);  // column offset of this pipe's TMEM block
   const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
   const int gr = qtile * kRows + r;
-  const bool row_ok = gr < p.rows_total;
+  const bool row_ok = pipe < nq && gr < p.rows_total;
   const int hq = hk * p.G + gr % p.G;
   const int u = min(gr / p.G, p.M);
   uint32_t anc_w[kMaxRows / 32];
@@ -317,8 +335,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         hi = __ldg(src + c + 8);
         if (rope) rope_rotate8(lo, hi, pos, p.rope.f, 8 * c);
       }
-      *reinterpret_cast<uint4*>(q_s + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
-      *reinterpret_cast<uint4*>(q_s + kRows * 128 + r * 128 + ((c ^ (r & 7)) << 4)) = hi;
+      *reinterpret_cast<uint4*>(q_pipe + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
+      *reinterpret_cast<uint4*>(q_pipe + kRows * 128 + r * 128 + ((c ^ (r & 7)) << 4)) = hi;
     }
     fence_async_smem();  // generic-proxy stores -> visible to the tensor core after the barrier
 #pragma unroll
@@ -327,14 +345,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   }
   if (warp == 1) {
     __syncwarp();  // tcgen05.alloc is warp-collective
-    tmem_alloc(&sh->tmem_base, kTmemCols);
+    tmem_alloc(&sh->tmem_base, kTmemCols * NQ);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t t_s0 = tmem, t_o = tmem + 128;
+  const uint32_t t_s0 = tmem + tq, t_o = tmem + tq + 128;  // this warp's pipe
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -378,7 +396,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && ntiles > 0) {
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
-      const uint32_t q_addr = smem_u32(q_s);
       bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
         const int s = i % k_stages, sb = i & 1;
@@ -388,17 +405,20 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         }
         tc_fence_after();
         const uint32_t k_addr = smem_u32(k_ring + s * kTileBytes);
+        for (int q = 0; q < nq; ++q) {  // S_q = Q_q K^T, every pipe on the same K tile
+          const uint32_t q_addr = smem_u32(q_s + q * kQBytes);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
-          const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
-          mma_ss(t_s0 + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
+            const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
+            mma_ss(tmem + q * kTmemCols + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+          }
+          tc_commit(&sh->s_full[q][sb]);
         }
         tc_commit(&sh->k_empty[s]);
-        tc_commit(&sh->s_full[sb]);
-        if (i >= 1 && !issue_pv(sh, v_ring, t_s0, t_o, i - 1, v_stages, lim)) to = true;
+        if (i >= 1 && !issue_pv(sh, v_ring, tmem, nq, i - 1, v_stages, lim)) to = true;
       }
-      if (!to && !issue_pv(sh, v_ring, t_s0, t_o, ntiles - 1, v_stages, lim)) to = true;
+      if (!to && !issue_pv(sh, v_ring, tmem, nq, ntiles - 1, v_stages, lim)) to = true;
       if (to) atomicExch(&sh->timed_out, 1);
       // Every MMA issued so far retires before TMEM and shared memory are
       // released, also when a softmax warp gave up before reading the last O.
@@ -412,13 +432,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   float m = -INFINITY, l = 0.f;
   bool have = false;
   const bool warp_live = __any_sync(0xffffffffu, row_ok);  // some row of this warp is real
-  if (warp >= 2) {
+  if (warp >= 2 && pipe < nq) {
     bool to = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1;
       // every wait that gates a TMEM access is decided for the whole warp: the
       // tcgen05.ld / tcgen05.st that follow are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[sb], (i >> 1) & 1, lim))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[pipe][sb], (i >> 1) & 1, lim))) {
         to = true;
         break;
       }
@@ -457,7 +477,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
         const bool scale_o = grow && m != -INFINITY;
         if (__any_sync(0xffffffffu, scale_o)) {
           // O holds earlier tiles: rescale once PV_{i-1} has landed
-          if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, lim))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&sh->o_ready[pipe][(i - 1) & 1], ((i - 1) >> 1) & 1, lim))) {
             to = true;
             break;
           }
@@ -509,7 +529,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       }
       // past the end of the key range the V rows may hold anything: zero them
       const int kend = N - key0;
-      if (kend < kKeyTile) {
+      if (kend < kKeyTile && pipe == 0) {  // pipe 0 zeroes; every PV on this tile waits for it
         uint8_t* vt = v_ring + (i % v_stages) * kTileBytes;
         if (!__all_sync(0xffffffffu, mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1, lim))) {
           to = true;  // V_i must have landed before its rows are overwritten
@@ -525,12 +545,12 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh->p_full[sb]);
+      if (lane == 0) mbar_arrive(&sh->p_full[pipe][sb]);
     }
     if (to) atomicExch(&sh->timed_out, 1);
     have = __all_sync(0xffffffffu, ntiles > 0 && !to && warp_live);
     if (ntiles > 0 && !to) {
-      if (!mbar_wait(&sh->o_ready[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, lim)) {
+      if (!mbar_wait(&sh->o_ready[pipe][(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, lim)) {
         atomicExch(&sh->timed_out, 1);
         have = false;
       }
@@ -541,7 +561,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       // normalised bf16 row -> smem (the Q tile is dead once the last MMA is done),
       // then the four warps copy whole rows out with coalesced 16-byte stores
       const float inv = (have && valid && l > 0.f) ? 1.f / l : 0.f;
-      uint8_t* ost = q_s;  // [128 rows][256 B], 16-byte chunks rotated by row
+      uint8_t* ost = q_pipe;  // [128 rows][256 B], 16-byte chunks rotated by row
       if (warp_live) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -565,9 +585,9 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
           }
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + pipe) : "memory");  // the four softmax warps of this pipe
       const int rows = min(kRows, p.rows_total - qtile * kRows);
-      const int t = (warp - 2) * 32 + lane;
+      const int t = ((warp - 2) & 3) * 32 + lane;
       for (int idx = t; idx < rows * 16; idx += 128) {
         const int rr = idx >> 4, chunk = idx & 15;
         const int g2 = qtile * kRows + rr;
@@ -585,12 +605,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     // share of the rows from the other splits' records.
     cg::cluster_group cluster = cg::this_cluster();
     const int ns = p.nsplit;
-    const int unit = bh * gridDim.y + qtile;
-    // workspace records are chunk-major ([32 float4 chunks][128 rows]) so that a
-    // warp's 32 rows write, and read back, 512 contiguous bytes
-    float4* ws_o = reinterpret_cast<float4*>(p.ws) + (size_t)unit * ns * 32 * kRows;
-    float2* ws_ml = reinterpret_cast<float2*>(p.ws + (size_t)gridDim.z * gridDim.y * ns * kRows * 128) +
-                    (size_t)unit * ns * kRows;
+    // records per query tile (unit = (sequence, kv head, query tile)); chunk-major
+    // ([32 float4 chunks][128 rows]) so that a warp's 32 rows write, and read
+    // back, 512 contiguous bytes
+    const size_t n_units = (size_t)gridDim.z * tiles_q;
+    auto rec_o = [&](int qt) {
+      return reinterpret_cast<float4*>(p.ws) + ((size_t)bh * tiles_q + qt) * ns * 32 * kRows;
+    };
+    auto rec_ml = [&](int qt) {
+      return reinterpret_cast<float2*>(p.ws + n_units * ns * kRows * 128) + ((size_t)bh * tiles_q + qt) * ns * kRows;
+    };
+    float4* ws_o = rec_o(qtile);
+    float2* ws_ml = rec_ml(qtile);
     if (warp >= 2 && warp_live) {
       float4* dst = ws_o + (size_t)split * 32 * kRows + r;
 #pragma unroll
@@ -622,21 +648,26 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
     tc_fence_before();
     cluster.sync();  // every split's record is written
     const int rank = (int)cluster.block_rank();
-    const int rows = min(kRows, p.rows_total - qtile * kRows);  // real rows of this tile
-    // rank j merges chunks [q_lo, q_hi) of every real row; consecutive threads take
-    // consecutive rows, so each split's record is read with coalesced loads
+    // rank j merges chunks [q_lo, q_hi) of every real row of every query tile of
+    // the CTA; consecutive threads take consecutive rows, so each split's
+    // record is read with coalesced loads
     const int q_lo = rank * 32 / ns, q_hi = (rank + 1) * 32 / ns;
+    for (int mq = 0; mq < nq; ++mq) {
+    const int mtile = qtile0 + mq;
+    const int rows = min(kRows, p.rows_total - mtile * kRows);  // real rows of this tile
+    const float4* mo = rec_o(mtile);
+    const float2* mml = rec_ml(mtile);
     for (int idx = threadIdx.x; idx < (q_hi - q_lo) * rows; idx += blockDim.x) {
       const int rr = idx % rows;
       const int q = q_lo + idx / rows;
-      const int g2 = qtile * kRows + rr;
+      const int g2 = mtile * kRows + rr;
       float2 ml[kMaxSplit_tc];
       float4 oj[kMaxSplit_tc];
 #pragma unroll
       for (int j = 0; j < kMaxSplit_tc; ++j) {
         if (j < ns) {
-          ml[j] = __ldcg(ws_ml + (size_t)j * kRows + rr);
-          oj[j] = __ldcg(ws_o + ((size_t)j * 32 + q) * kRows + rr);
+          ml[j] = __ldcg(mml + (size_t)j * kRows + rr);
+          oj[j] = __ldcg(mo + ((size_t)j * 32 + q) * kRows + rr);
         } else {
           ml[j] = make_float2(-INFINITY, 0.f);
           oj[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -664,6 +695,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
       pk.y = pack_bf16x2(a.z * inv, a.w * inv);
       *reinterpret_cast<uint2*>(p.out + orow + q * 4) = pk;
     }
+    }
   } else {
     tc_fence_before();
     __syncthreads();
@@ -671,7 +703,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) tree_attn_tc_kernel(const __gri
   if (warp == 1) {
     __syncwarp();  // tcgen05.dealloc is warp-collective
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols * NQ);
   }
   if (threadIdx.x == 0 && (sh->timed_out || !aligned_ok)) atomicOr(&p.status[b], kSeqTimeout);
   if (threadIdx.x == 0 && (broken_promise || sl < 0)) atomicOr(&p.status[b], kSeqBadGeometry);
@@ -686,27 +718,41 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rows_total = (Hq / Hkv) * (M + 1);
   lp.tiles_q = (rows_total + kRows - 1) / kRows;
-  const int64_t units = (int64_t)B * Hkv * lp.tiles_q;
+  // Two query tiles per CTA whenever a (sequence, kv head) has two or more:
+  // every K/V tile brought into shared memory then serves both, which halves
+  // the K/V traffic from L2 (the tensor-bound shapes read each K/V byte once
+  // per query tile, and that traffic, not the tensor cores, bounds them).
+  lp.nq = (TV_TC_PAIR && lp.tiles_q >= 2) ? 2 : 1;
+  const int grid_y = (lp.tiles_q + lp.nq - 1) / lp.nq;
+  const int64_t units = (int64_t)B * Hkv * lp.tiles_q;  // query tiles (workspace records)
+  const int64_t ctas_per_split = (int64_t)B * Hkv * grid_y;
   const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
   // Split the key range only while the query tiles alone leave SMs idle: a
-  // split adds a merge, and past one CTA per SM it adds a partial second wave.
-  int ns = units >= sms ? 1
-                        : (int)std::min<int64_t>(kMaxSplit_tc,
-                                                 std::max<int64_t>(1, ((int64_t)TV_TC_SPLIT_FACTOR * sms) / units));
+  // split adds a merge, and past the resident CTAs it adds a partial wave.
+  const int64_t cap = lp.nq == 2 ? sms : (int64_t)TV_TC_SPLIT_FACTOR * sms;  // CTAs that fit at once
+  int ns = ctas_per_split >= sms ? 1
+                                 : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, cap / ctas_per_split));
   ns = std::min(ns, key_tiles);
   lp.tiles_per_split = (key_tiles + ns - 1) / ns;
   lp.nsplit = (key_tiles + lp.tiles_per_split - 1) / lp.tiles_per_split;
-  // Deepest ring that keeps the grid resident: two CTAs per SM when the grid
-  // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
-  // never waits on a CTA that is itself waiting), else one CTA per SM.
-  const int64_t ctas = units * lp.nsplit;
-  const bool two_per_sm = !TV_TC_FORCE_SOLO && (!TV_TC_ONE_PER_SM || ctas > sms);
-  // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
-  // one CTA per SM: K ring 3, V ring up to 6
-  lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
-  lp.v_stages = two_per_sm ? 3 : std::min(TV_TC_V_RING_SOLO, std::max(2, lp.tiles_per_split));
-  const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
-  lp.smem = std::max(smem_min, kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem));
+  if (lp.nq == 2) {
+    // one CTA per SM (all 512 TMEM columns): deep rings
+    lp.stages = std::min(4, std::max(2, lp.tiles_per_split));
+    lp.v_stages = std::min(5, std::max(2, lp.tiles_per_split));
+    lp.smem = 2 * (size_t)kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem);
+  } else {
+    // Deepest ring that keeps the grid resident: two CTAs per SM when the grid
+    // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
+    // never waits on a CTA that is itself waiting), else one CTA per SM.
+    const int64_t ctas = ctas_per_split * lp.nsplit;
+    const bool two_per_sm = !TV_TC_FORCE_SOLO && (!TV_TC_ONE_PER_SM || ctas > sms);
+    // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
+    // one CTA per SM: deeper rings
+    lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
+    lp.v_stages = two_per_sm ? 3 : std::min(TV_TC_V_RING_SOLO, std::max(2, lp.tiles_per_split));
+    const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
+    lp.smem = std::max(smem_min, kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem));
+  }
   lp.ws_bytes = lp.nsplit > 1 ? (size_t)units * lp.nsplit * kRows * (128 + 2) * sizeof(float) : 0;
   return TV_OK;
 }
@@ -717,15 +763,19 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   p.nsplit = lp.nsplit;
   p.stages = lp.stages;
   p.v_stages = lp.v_stages;
-  cudaError_t e = cudaFuncSetAttribute(tree_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
+  if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
+  const int grid_y = (lp.tiles_q + lp.nq - 1) / lp.nq;
+  dim3 grid(lp.nsplit, grid_y, p.B * p.Hkv);
+  auto kern = lp.nq == 2 ? tree_attn_tc_kernel<2> : tree_attn_tc_kernel<1>;
+  const int threads = 64 + 128 * lp.nq;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
   if (e != cudaSuccess) return record_cuda_error(e);
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tree_attn_tc_kernel, kTcThreads, lp.smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, lp.smem);
   if (e != cudaSuccess) return record_cuda_error(e);
-  if (occ > 2 || occ < 1) return TV_ERR_UNSUPPORTED;
-  if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
-  dim3 grid(lp.nsplit, lp.tiles_q, p.B * p.Hkv);
-  return launch(tree_attn_tc_kernel, grid, dim3(kTcThreads), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
+  // TMEM: 256 columns per query tile; never more CTAs on an SM than 512 columns hold
+  if (occ < 1 || occ * lp.nq > 2) return TV_ERR_UNSUPPORTED;
+  return launch(kern, grid, dim3(threads), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
 }  // namespace tv
