@@ -56,9 +56,10 @@ namespace cg = cooperative_groups;
 #endif
 //   TV_TC_FORCE_SOLO    1: one CTA per SM (deep rings) even for grids of
 //                       several waves
-//   TV_TC_PAIR          1: two query tiles per CTA when a unit has two or more
+//   TV_TC_PAIR          1: two query tiles per CTA when a unit has two or more (off:
+//                       measured slower)
 #ifndef TV_TC_PAIR
-#define TV_TC_PAIR 1
+#define TV_TC_PAIR 0
 #endif
 #ifndef TV_TC_FORCE_SOLO
 #define TV_TC_FORCE_SOLO 0
@@ -718,10 +719,11 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int rows_total = (Hq / Hkv) * (M + 1);
   lp.tiles_q = (rows_total + kRows - 1) / kRows;
-  // Two query tiles per CTA whenever a (sequence, kv head) has two or more:
-  // every K/V tile brought into shared memory then serves both, which halves
-  // the K/V traffic from L2 (the tensor-bound shapes read each K/V byte once
-  // per query tile, and that traffic, not the tensor cores, bounds them).
+  // Two query tiles per CTA (TV_TC_PAIR) when a (sequence, kv head) has two or
+  // more: every K/V tile brought into shared memory then serves both, halving
+  // the K/V traffic from L2.  Measured slower on B200 (b32gqa 252 vs 162 us,
+  // stress 2.41 vs 1.63 ms per launch: one CTA per SM with two pipes loses to
+  // two CTAs per SM with one pipe each), so it is off by default.
   lp.nq = (TV_TC_PAIR && lp.tiles_q >= 2) ? 2 : 1;
   const int grid_y = (lp.tiles_q + lp.nq - 1) / lp.nq;
   const int64_t units = (int64_t)B * Hkv * lp.tiles_q;  // query tiles (workspace records)
