@@ -89,6 +89,7 @@ inline bool encode_kv_map(CUtensorMap* map, const void* base, int BH, int64_t S_
 // Tensor-core (tcgen05) path for head dim 128; defined in attention_tc.cu.
 struct TcPlan {
   int tiles_q, nq, nsplit, tiles_per_split, stages, v_stages;  // nq: query tiles per CTA
+  int per_sm;  // CTAs the plan sizes to be resident on one SM
   size_t smem, ws_bytes;
 };
 tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan& plan);

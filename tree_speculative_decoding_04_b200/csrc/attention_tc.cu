@@ -10,7 +10,9 @@
 // (sequence, kv head) and one split of that sequence's key range.  The splits
 // of a query tile form a thread-block cluster: each writes its partial (max,
 // sum, O) to a workspace in L2, the cluster barrier orders the writes, and each
-// CTA then merges 1/nsplit of the output columns.
+// CTA then merges 1/nsplit of the output columns.  (Keeping the partials in
+// each CTA's shared memory and merging over distributed shared memory gave the
+// same bits and measured no faster on B200.)
 // Warp roles (192 threads):
 //   warp 0      TMA producer: 64-key K tiles and V tiles into two separate smem
 //               rings -- a K slot is freed as soon as S = QK^T has read it, a V
@@ -70,6 +72,11 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_V_RING_SOLO
 #define TV_TC_V_RING_SOLO 6
 #endif
+//   TV_TC_LONGEST_FIRST  1: grids of more than one wave start their (sequence,
+//                       kv head) blocks longest prefix first
+#ifndef TV_TC_LONGEST_FIRST
+#define TV_TC_LONGEST_FIRST 1
+#endif
 
 namespace tv {
 namespace {
@@ -96,6 +103,69 @@ struct TcSmem {
   uint32_t tmem_base;
   int timed_out;
 };
+
+// The batch row that the `rank`-th (sequence, kv head) block of the grid
+// serves, with its cache slot, geometry and status.  Rows are taken longest
+// prefix first (ties in row order): the block scheduler starts blocks in grid
+// order, so the longest units start first and the last wave is made of short
+// ones (longest-processing-time-first list scheduling); in plain row order a
+// long sequence that happens to come last leaves most SMs idle at the end.
+// For B <= 32 lane i of the calling warp loads row i's slot, kv_len, kv_start
+// and status in one round trip, the rows are ranked with shuffles and the
+// chosen row's values are shuffled out; every lane gets the same answer.
+// Larger batches, and grids that start all at once (LF = false: the order
+// cannot matter there), keep row order.  Warp-collective: call with all lanes
+// active.
+struct RowGeo {
+  int b;         // batch row
+  int sl;        // cache slot (-1: outside the pool)
+  int32_t ks;    // kv_start of the slot (0 when sl < 0)
+  int32_t kl;    // kv_len of the slot (0 when sl < 0)
+  int32_t st;    // status of the row
+  int32_t lane_len;  // this lane's row length (-1 past B or outside the pool; 0 for B > 32)
+};
+
+template <bool LF>
+__device__ __forceinline__ RowGeo row_of_rank(const AttnParams& p, int rank) {
+  RowGeo g;
+  if (!LF || p.B > 32) {
+    g.b = rank;
+    g.sl = cache_slot(p.slot, rank, p.n_slots);
+    g.ks = g.sl >= 0 ? __ldcg(p.kv_start + g.sl) : 0;
+    g.kl = g.sl >= 0 ? __ldcg(p.kv_len + g.sl) : 0;
+    g.st = __ldcg(p.status + rank);
+    g.lane_len = 0;
+    return g;
+  }
+  const int lane = threadIdx.x & 31;
+  int s = -1;
+  int32_t len = -1, ks = 0, st = 0;
+  if (lane < p.B) {
+    s = cache_slot(p.slot, lane, p.n_slots);
+    st = __ldcg(p.status + lane);
+    if (s >= 0) {
+      len = __ldcg(p.kv_len + s);
+      ks = __ldcg(p.kv_start + s);
+    }
+  }
+  // rank of this lane's row: rows that are longer, or as long and earlier
+  int r = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int32_t lj = __shfl_sync(0xffffffffu, len, j);
+    r += (j < p.B && (lj > len || (lj == len && j < lane))) ? 1 : 0;
+  }
+  const unsigned m = __ballot_sync(0xffffffffu, lane < p.B && r == rank);
+  const int src = m ? __ffs(m) - 1 : 0;  // (len, -row) is a strict order: exactly one lane matches
+  g.b = m ? src : rank;
+  g.sl = __shfl_sync(0xffffffffu, s, src);
+  g.ks = __shfl_sync(0xffffffffu, ks, src);
+  g.kl = __shfl_sync(0xffffffffu, len, src);
+  g.st = __shfl_sync(0xffffffffu, st, src);
+  if (g.sl < 0) g.ks = g.kl = 0;
+  g.lane_len = len;
+  return g;
+}
 
 // bits [start, start + 64) of an ancestor row (bit t = tree row t); rows outside
 // [0, 32 * 8) read as 0, so a window that starts inside the prefix is fine.
@@ -137,8 +207,11 @@ __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t t
 
 // NQ query tiles per CTA share every K/V tile (NQ = 2: 8 softmax warps, all 512
 // TMEM columns, one CTA per SM); the query tiles of a (sequence, kv head) are
-// blockIdx.y * NQ + q.
-template <int NQ>
+// blockIdx.y * NQ + q.  LF: blocks take their batch row longest prefix first
+// (a separate instance: the ranking code, even when skipped at run time, cost
+// single-wave grids about 4 us per launch on B200 through code generation at
+// the register limit).
+template <int NQ, bool LF>
 __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                         const __grid_constant__ AttnParams p) {
@@ -161,8 +234,8 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   const int qtile0 = blockIdx.y * NQ;                  // first query tile of this CTA
   const int nq = min(NQ, tiles_q - qtile0);            // query tiles present (the last CTA may have fewer)
   const int bh = blockIdx.z;
-  const int b = bh / p.Hkv;
-  const int hk = bh - b * p.Hkv;
+  const int hk = bh % p.Hkv;
+  const int rank = bh / p.Hkv;  // the block's place in the longest-first row order
 
   if (threadIdx.x == 0) {
     sh->timed_out = 0;
@@ -232,72 +305,75 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   // limit of the pipeline waits; the waits that drain copies or MMAs in flight
   // before the CTA exits always keep the full limit
   const uint64_t lim = p.wait_limit_ns;
-  int32_t ks = 0, kl = 0;
-  int sl = -1;                 // cache slot of this batch row (-1: outside the pool)
+  // Warp 0 reads the row order and the geometry before the grid dependency
+  // (one round trip); the other warps read them after it only.
+  RowGeo pre{rank, -1, 0, 0, 0, 0};
   int npre_k = 0, npre_v = 0;  // tiles requested before the grid dependency
-  if (prefix_ready) {
-    sl = cache_slot(p.slot, b, p.n_slots);
-    if (sl >= 0) {
-      ks = __ldcg(p.kv_start + sl);
-      kl = __ldcg(p.kv_len + sl);
-    }
-    if (sl >= 0 && aligned_ok && geometry_ok(ks, kl, p.M, p.S_cap)) {
-      int k_lo_pre, nt_pre;
-      split_range(kl, k_lo_pre, nt_pre);
-      const int n_prefix = max(0, min(nt_pre, (kl - k_lo_pre) / kKeyTile));  // tiles wholly inside the prefix
-      npre_k = min(n_prefix, k_stages);
-      npre_v = min(n_prefix, v_stages);
-      if (warp == 0 && lane == 0)  // the thread that initialised the barriers
-        for (int i = 0; i < max(npre_k, npre_v); ++i) {
-          if (i < npre_k) issue_k(i, ks, k_lo_pre, sl * p.Hkv + hk);
-          if (i < npre_v) issue_v(i, ks, k_lo_pre, sl * p.Hkv + hk);
-        }
-    }
-  } else if (warp == 0 && lane == 0) {
-    const int sl_h = p.slot ? __ldcg(p.slot + b) : b;
-    if (sl_h >= 0 && sl_h < p.n_slots) {
-      const int32_t ks_h = __ldcg(p.kv_start + sl_h), kl_h = __ldcg(p.kv_len + sl_h);
-      if (geometry_ok(ks_h, kl_h, p.M, p.S_cap)) {
-        int k_lo_h, nt_h;
-        split_range(kl_h, k_lo_h, nt_h);
-        const int nt = min(kPrefetchTiles, nt_h);
-        for (int i = 0; i < nt; ++i) {
-          const int row = ks_h + k_lo_h + i * kKeyTile;
-          if (p.kv_4d) {
-            tma_prefetch_4d(&tmk, 0, row, 0, sl_h * p.Hkv + hk);
-            tma_prefetch_4d(&tmv, 0, row, 0, sl_h * p.Hkv + hk);
-          } else {
-            tma_prefetch_3d(&tmk, 0, row, sl_h * p.Hkv + hk);
-            tma_prefetch_3d(&tmk, 64, row, sl_h * p.Hkv + hk);
-            tma_prefetch_3d(&tmv, 0, row, sl_h * p.Hkv + hk);
-            tma_prefetch_3d(&tmv, 64, row, sl_h * p.Hkv + hk);
+  if (warp == 0) {
+    pre = row_of_rank<LF>(p, rank);
+    if (prefix_ready) {
+      if (pre.sl >= 0 && aligned_ok && geometry_ok(pre.ks, pre.kl, p.M, p.S_cap)) {
+        int k_lo_pre, nt_pre;
+        split_range(pre.kl, k_lo_pre, nt_pre);
+        const int n_prefix = max(0, min(nt_pre, (pre.kl - k_lo_pre) / kKeyTile));  // tiles wholly inside the prefix
+        npre_k = min(n_prefix, k_stages);
+        npre_v = min(n_prefix, v_stages);
+        if (lane == 0)  // the thread that initialised the barriers
+          for (int i = 0; i < max(npre_k, npre_v); ++i) {
+            if (i < npre_k) issue_k(i, pre.ks, k_lo_pre, pre.sl * p.Hkv + hk);
+            if (i < npre_v) issue_v(i, pre.ks, k_lo_pre, pre.sl * p.Hkv + hk);
           }
+      }
+    } else if (lane == 0 && pre.sl >= 0 && geometry_ok(pre.ks, pre.kl, p.M, p.S_cap)) {
+      int k_lo_h, nt_h;
+      split_range(pre.kl, k_lo_h, nt_h);
+      const int nt = min(kPrefetchTiles, nt_h);
+      for (int i = 0; i < nt; ++i) {
+        const int row = pre.ks + k_lo_h + i * kKeyTile;
+        if (p.kv_4d) {
+          tma_prefetch_4d(&tmk, 0, row, 0, pre.sl * p.Hkv + hk);
+          tma_prefetch_4d(&tmv, 0, row, 0, pre.sl * p.Hkv + hk);
+        } else {
+          tma_prefetch_3d(&tmk, 0, row, pre.sl * p.Hkv + hk);
+          tma_prefetch_3d(&tmk, 64, row, pre.sl * p.Hkv + hk);
+          tma_prefetch_3d(&tmv, 0, row, pre.sl * p.Hkv + hk);
+          tma_prefetch_3d(&tmv, 64, row, pre.sl * p.Hkv + hk);
         }
       }
     }
   }
-  if (warp >= 2) {
+  // the query rows are warmed in L2 when the row is known without a load
+  if (warp >= 2 && (!LF || p.B > 32)) {
     const int gr_h = (qtile0 + ((warp - 2) >> 2)) * kRows + (warp & 3) * 32 + lane;
     if (gr_h < p.rows_total) {
-      const uint16_t* qr = p.q + (((int64_t)b * (p.M + 1) + gr_h / p.G) * p.Hq + hk * p.G + gr_h % p.G) * 128;
+      const uint16_t* qr =
+          p.q + (((int64_t)rank * (p.M + 1) + gr_h / p.G) * p.Hq + hk * p.G + gr_h % p.G) * 128;
       prefetch_l2(qr);
       prefetch_l2(qr + 64);
     }
   }
   pdl_wait_primary();
   pdl_launch_dependents();
-  // The slot and the geometry are read again after the dependency: if the
-  // caller's promise did not hold (they changed), the sequence is flagged
-  // instead of computed.
-  const int sl_now = cache_slot(p.slot, b, p.n_slots);
-  const int32_t ks_now = sl_now >= 0 ? p.kv_start[sl_now] : 0, kl_now = sl_now >= 0 ? p.kv_len[sl_now] : 0;
-  const bool broken_promise = prefix_ready && (sl_now != sl || ks_now != ks || kl_now != kl);
-  sl = sl_now;
-  ks = ks_now;
-  kl = kl_now;
+  // The row order, the slot and the geometry are read again after the
+  // dependency (final values, the same for every warp).  Without
+  // TV_ATTN_PREFIX_READY warp 0's early read served only prefetches.  With it,
+  // if the caller's promise did not hold (they changed), the sequence is
+  // flagged instead of computed; a changed length may also have changed the
+  // row order, which CTAs that read early no longer share with the others, so
+  // then every row of the batch is flagged.
+  const RowGeo g = row_of_rank<LF>(p, rank);
+  const int b = g.b;
+  const int sl = g.sl;
+  const int32_t ks = g.ks, kl = g.kl;
+  bool order_changed = false, broken_promise = false;
+  if (prefix_ready) {  // uniform over the CTA
+    const bool changed_w = warp == 0 && __any_sync(0xffffffffu, g.lane_len != pre.lane_len);
+    order_changed = __syncthreads_or(changed_w) != 0;
+    broken_promise = __syncthreads_or(warp == 0 && (changed_w || g.b != pre.b || g.sl != pre.sl ||
+                                                    g.ks != pre.ks || g.kl != pre.kl)) != 0;
+  }
   const int zc = sl * p.Hkv + hk;  // tensor-map row block of this (slot, kv head)
-  const bool valid = aligned_ok && sl >= 0 && !broken_promise && p.status[b] == 0 &&
-                     geometry_ok(ks, kl, p.M, p.S_cap);
+  const bool valid = aligned_ok && sl >= 0 && !broken_promise && g.st == 0 && geometry_ok(ks, kl, p.M, p.S_cap);
   const int N = kl + p.M + 1;
   int k_lo = 0, nt_geo = 0;
   split_range(kl, k_lo, nt_geo);
@@ -708,6 +784,8 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   }
   if (threadIdx.x == 0 && (sh->timed_out || !aligned_ok)) atomicOr(&p.status[b], kSeqTimeout);
   if (threadIdx.x == 0 && (broken_promise || sl < 0)) atomicOr(&p.status[b], kSeqBadGeometry);
+  if (threadIdx.x == 0 && order_changed)
+    for (int i = 0; i < p.B; ++i) atomicOr(&p.status[i], kSeqBadGeometry);
 }
 
 }  // namespace
@@ -729,8 +807,8 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
   const int64_t units = (int64_t)B * Hkv * lp.tiles_q;  // query tiles (workspace records)
   const int64_t ctas_per_split = (int64_t)B * Hkv * grid_y;
   const int key_tiles = (int)std::max<int64_t>(1, (S_cap + kKeyTile - 1) / kKeyTile);
-  // Split the key range only while the query tiles alone leave SMs idle: a
-  // split adds a merge, and past the resident CTAs it adds a partial wave.
+  // Split the key range while the query tiles alone leave SMs idle: a split
+  // adds a merge, and past the resident CTAs it adds a partial wave.
   const int64_t cap = lp.nq == 2 ? sms : (int64_t)TV_TC_SPLIT_FACTOR * sms;  // CTAs that fit at once
   int ns = ctas_per_split >= sms ? 1
                                  : (int)std::min<int64_t>(kMaxSplit_tc, std::max<int64_t>(1, cap / ctas_per_split));
@@ -742,12 +820,14 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
     lp.stages = std::min(4, std::max(2, lp.tiles_per_split));
     lp.v_stages = std::min(5, std::max(2, lp.tiles_per_split));
     lp.smem = 2 * (size_t)kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem);
+    lp.per_sm = 1;
   } else {
     // Deepest ring that keeps the grid resident: two CTAs per SM when the grid
     // needs it (each then holds 256 of the 512 TMEM columns, so an allocation
     // never waits on a CTA that is itself waiting), else one CTA per SM.
     const int64_t ctas = ctas_per_split * lp.nsplit;
     const bool two_per_sm = !TV_TC_FORCE_SOLO && (!TV_TC_ONE_PER_SM || ctas > sms);
+    lp.per_sm = two_per_sm ? 2 : 1;
     // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
     // one CTA per SM: deeper rings
     lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
@@ -768,15 +848,32 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
   const int grid_y = (lp.tiles_q + lp.nq - 1) / lp.nq;
   dim3 grid(lp.nsplit, grid_y, p.B * p.Hkv);
-  auto kern = lp.nq == 2 ? tree_attn_tc_kernel<2> : tree_attn_tc_kernel<1>;
   const int threads = 64 + 128 * lp.nq;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // The instance: blocks in longest-first order only when not every block
+  // starts at once (more blocks than the plan's resident CTAs) and the batch is
+  // small enough to rank in one warp.
+  auto occupancy = [&](auto kern, int& occ) {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lp.smem);
+    if (err != cudaSuccess) return err;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, lp.smem);
+  };
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, lp.smem);
+  e = lp.nq == 2 ? occupancy(tree_attn_tc_kernel<2, false>, occ) : occupancy(tree_attn_tc_kernel<1, false>, occ);
   if (e != cudaSuccess) return record_cuda_error(e);
+  const bool lf = TV_TC_LONGEST_FIRST && lp.nq == 1 && p.B > 1 && p.B <= 32 &&
+                  (int64_t)grid.x * grid.y * grid.z > (int64_t)lp.per_sm * sms;
+  if (lf) {
+    e = occupancy(tree_attn_tc_kernel<1, true>, occ);
+    if (e != cudaSuccess) return record_cuda_error(e);
+  }
   // TMEM: 256 columns per query tile; never more CTAs on an SM than 512 columns hold
   if (occ < 1 || occ * lp.nq > 2) return TV_ERR_UNSUPPORTED;
+  auto kern = lp.nq == 2 ? tree_attn_tc_kernel<2, false>
+                         : (lf ? tree_attn_tc_kernel<1, true> : tree_attn_tc_kernel<1, false>);
   return launch(kern, grid, dim3(threads), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
