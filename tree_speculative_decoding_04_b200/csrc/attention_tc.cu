@@ -77,6 +77,20 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_LONGEST_FIRST
 #define TV_TC_LONGEST_FIRST 1
 #endif
+//   TV_TC_Q_TMEM        1: the one-query-tile instance keeps Q in TMEM (the A
+//                       operand of S = Q K^T) and a single S buffer, so each
+//                       score MMA reads only its K tile from shared memory
+#ifndef TV_TC_Q_TMEM
+#define TV_TC_Q_TMEM 0
+#endif
+//   TV_TC_TILE_MAJOR    1: single-wave grids issue their blocks query-tile-major
+#ifndef TV_TC_TILE_MAJOR
+#define TV_TC_TILE_MAJOR 1
+#endif
+//   TV_TC_SPLIT_PRODUCER 1: two producer threads, one per K and V stream
+#ifndef TV_TC_SPLIT_PRODUCER
+#define TV_TC_SPLIT_PRODUCER 1
+#endif
 
 namespace tv {
 namespace {
@@ -185,14 +199,16 @@ __device__ __forceinline__ uint64_t anc_window(const uint32_t (&aw)[kMaxRows / 3
 // then release the V stage once every pipe has used it and publish each new
 // O.  Pipe q's TMEM block starts at column q * 256: S buffers at +0 / +64 (P_j
 // aliases S[j % 2]), O at +128.  Returns false if a P or V never arrived.
+// single_s: one S buffer per pipe (P_j at column 0, p_full[q][0] completes one
+// phase per tile).
 __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t tmem, int nq, int j, int v_stages,
-                                         uint64_t lim) {
+                                         uint64_t lim, bool single_s = false) {
   const uint32_t idesc_o = idesc_bf16(128, 128, 1);
-  const int sb = j & 1, s = j % v_stages;
+  const int sb = single_s ? 0 : (j & 1), s = j % v_stages;
   if (!mbar_wait(&sh->v_full[s], (j / v_stages) & 1, lim)) return false;
   const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
   for (int q = 0; q < nq; ++q) {
-    if (!mbar_wait(&sh->p_full[q][sb], (j >> 1) & 1, lim)) return false;
+    if (!mbar_wait(&sh->p_full[q][sb], single_s ? (j & 1) : ((j >> 1) & 1), lim)) return false;
     tc_fence_after();
     const uint32_t t_q = tmem + q * kTmemCols;
 #pragma unroll
@@ -207,17 +223,22 @@ __device__ __forceinline__ bool issue_pv(TcSmem* sh, uint8_t* v_ring, uint32_t t
 
 // NQ query tiles per CTA share every K/V tile (NQ = 2: 8 softmax warps, all 512
 // TMEM columns, one CTA per SM); the query tiles of a (sequence, kv head) are
-// blockIdx.y * NQ + q.  LF: blocks take their batch row longest prefix first
-// (a separate instance: the ranking code, even when skipped at run time, cost
-// single-wave grids about 4 us per launch on B200 through code generation at
-// the register limit).
-template <int NQ, bool LF>
+// blockIdx.y * NQ + q.  MW: the grid has more blocks than fit at once.  A
+// multi-wave grid is unit-major and, with TV_TC_LONGEST_FIRST, takes its batch
+// rows longest prefix first (a separate instance: the ranking code, even when
+// skipped at run time, cost single-wave grids about 4 us per launch on B200
+// through code generation at the register limit); a single-wave grid is
+// query-tile-major with TV_TC_TILE_MAJOR.  The host lays out the grid to match.
+template <int NQ, bool MW>
 __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
     tree_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                         const __grid_constant__ AttnParams p) {
   // The 128-byte-swizzled tiles need 1024-byte alignment.  The dynamic window
   // starts on such a boundary on this GPU; if it ever did not, every CTA treats
   // its sequence as failed (zero output, TV_SEQ_TIMEOUT) instead of computing.
+  // Q in TMEM and one S buffer (one query tile per CTA): TMEM S [0,64),
+  // Q [64,128), O [128,256); otherwise S0 [0,64), S1 [64,128), O [128,256)
+  constexpr bool kQT = NQ == 1 && TV_TC_Q_TMEM;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const bool aligned_ok = (smem_u32(smem_raw) & 1023u) == 0;
@@ -231,9 +252,18 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int tiles_q = (p.rows_total + kRows - 1) / kRows;
-  const int qtile0 = blockIdx.y * NQ;                  // first query tile of this CTA
+  // Grids of one wave (MW = false) are query-tile-major, grid (splits, units,
+  // query tiles): every unit's first tiles, then its second ones, and the last,
+  // often light tile (b32gqa: rows 128, 128, 16) of every unit at the end, so
+  // the CTAs that share an SM with another are light ones; every CTA of the
+  // wave starts at once, so the tiles of a unit still read its K/V together
+  // through L2.  Multi-wave grids stay unit-major, grid (splits, query tiles,
+  // units), so that the tiles of a unit run together.
+  constexpr bool kTileMajor = !MW && TV_TC_TILE_MAJOR;
+  constexpr bool LF = MW && TV_TC_LONGEST_FIRST;
+  const int qtile0 = (kTileMajor ? blockIdx.z : blockIdx.y) * NQ;  // first query tile of this CTA
   const int nq = min(NQ, tiles_q - qtile0);            // query tiles present (the last CTA may have fewer)
-  const int bh = blockIdx.z;
+  const int bh = kTileMajor ? blockIdx.y : blockIdx.z;
   const int hk = bh % p.Hkv;
   const int rank = bh / p.Hkv;  // the block's place in the longest-first row order
 
@@ -253,6 +283,7 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
         mbar_init(&sh->p_full[q][s], 4);
         mbar_init(&sh->o_ready[q][s], 1);
       }
+    mbar_init(&sh->q_ready, 4);  // the four softmax warps, once Q is in TMEM
     mbar_init(&sh->drain, 1);
     fence_mbar_init();
   }
@@ -382,10 +413,14 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   // The rest of the first ring's worth of K/V tiles and the Q tile are
   // requested before the TMEM allocation barrier, so their memory latency
   // overlaps the set-up.
-  if (warp == 0 && lane == 0)
+  // (lane 0 requests the K tiles, lane 1 the V tiles: the copies one thread
+  // issues are processed one after another, about 59 GB/s per issuing thread
+  // from L2 on B200, so two issuing threads keep K tiles from queueing behind
+  // V tiles)
+  if (warp == 0 && lane < (TV_TC_SPLIT_PRODUCER ? 2 : 1))
     for (int i = 0; i < min(ntiles, max(k_stages, v_stages)); ++i) {
-      if (i < k_stages && i >= npre_k) issue_k(i, ks, k_lo, zc);
-      if (i < v_stages && i >= npre_v) issue_v(i, ks, k_lo, zc);
+      if (lane == 0 && i < k_stages && i >= npre_k) issue_k(i, ks, k_lo, zc);
+      if (lane == (TV_TC_SPLIT_PRODUCER ? 1 : 0) && i < v_stages && i >= npre_v) issue_v(i, ks, k_lo, zc);
     }
   const int pipe = warp >= 2 ? (warp - 2) >> 2 : 0;  // query pipe of a softmax warp
   const int qtile = qtile0 + pipe;
@@ -433,45 +468,100 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      // K_i waits for S_{i-k_stages} to finish, V_i for PV_{i-v_stages}; both
-      // complete in the order this loop issues, so it never blocks early
+    // K_i waits for S_{i-k_stages} to finish, V_i for PV_{i-v_stages}; each
+    // stream completes in the order it is issued, so a wait never blocks early.
+    // Lane 0 streams K and lane 1 streams V (with a single producer, lane 0
+    // streams both, interleaved).
+    constexpr bool kSplit = TV_TC_SPLIT_PRODUCER != 0;
+    if (lane < (kSplit ? 2 : 1)) {
       bool to = false;
-      // the first ring's worth is already requested (or, for a sequence found
-      // invalid after the grid dependency, only the tiles requested before it)
-      int k_issued = ntiles > 0 ? min(ntiles, k_stages) : npre_k;
-      int v_issued = ntiles > 0 ? min(ntiles, v_stages) : npre_v;
-      for (int i = 0; i < ntiles && !to; ++i) {
-        if (i >= k_stages) {
-          if (!mbar_wait(&sh->k_empty[i % k_stages], ((i / k_stages) - 1) & 1, lim)) {
-            to = true;
-            break;
+      for (int st = 0; st < 2; ++st) {
+        if (kSplit && st != lane) continue;
+        const bool is_k = st == 0;
+        const int stages = is_k ? k_stages : v_stages;
+        uint64_t* full = is_k ? sh->k_full : sh->v_full;
+        uint64_t* empty = is_k ? sh->k_empty : sh->v_empty;
+        // the first ring's worth is already requested (or, for a sequence found
+        // invalid after the grid dependency, only the tiles requested before it)
+        int issued = ntiles > 0 ? min(ntiles, stages) : (is_k ? npre_k : npre_v);
+        if (kSplit) {
+          for (int i = stages; i < ntiles && !to; ++i) {
+            if (!mbar_wait(&empty[i % stages], ((i / stages) - 1) & 1, lim)) {
+              to = true;
+              break;
+            }
+            if (is_k)
+              issue_k(i, ks, k_lo, zc);
+            else
+              issue_v(i, ks, k_lo, zc);
+            ++issued;
           }
-          issue_k(i, ks, k_lo, zc);
-          ++k_issued;
-        }
-        if (i >= v_stages) {
-          if (!mbar_wait(&sh->v_empty[i % v_stages], ((i / v_stages) - 1) & 1, lim)) {
-            to = true;
-            break;
+        } else if (is_k) {
+          // one thread, K and V interleaved tile by tile
+          int v_issued = ntiles > 0 ? min(ntiles, v_stages) : npre_v;
+          for (int i = 0; i < ntiles && !to; ++i) {
+            if (i >= k_stages) {
+              if (!mbar_wait(&sh->k_empty[i % k_stages], ((i / k_stages) - 1) & 1, lim)) {
+                to = true;
+                break;
+              }
+              issue_k(i, ks, k_lo, zc);
+              ++issued;
+            }
+            if (i >= v_stages) {
+              if (!mbar_wait(&sh->v_empty[i % v_stages], ((i / v_stages) - 1) & 1, lim)) {
+                to = true;
+                break;
+              }
+              issue_v(i, ks, k_lo, zc);
+              ++v_issued;
+            }
           }
-          issue_v(i, ks, k_lo, zc);
-          ++v_issued;
+          for (int i = max(0, v_issued - v_stages); i < v_issued; ++i)
+            mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1);
         }
+        // Every copy issued must land before the CTA's shared memory is
+        // released, whether or not a consumer waited for it (a consumer that
+        // gave up, or a sequence found invalid, leaves copies unconsumed).  The
+        // last issued tile of each slot decides, so one wait per slot suffices.
+        for (int i = max(0, issued - stages); i < issued; ++i) mbar_wait(&full[i % stages], (i / stages) & 1);
+        if (!kSplit) break;  // the single producer handled V above
       }
       if (to) atomicExch(&sh->timed_out, 1);
-      // Every copy this thread issued must land before the CTA's shared memory
-      // is released, whether or not a consumer waited for it (a consumer that
-      // gave up, or a sequence found invalid, leaves copies unconsumed).  The
-      // last issued tile of each slot decides, so one wait per slot suffices.
-      for (int i = max(0, k_issued - k_stages); i < k_issued; ++i)
-        mbar_wait(&sh->k_full[i % k_stages], (i / k_stages) & 1);
-      for (int i = max(0, v_issued - v_stages); i < v_issued; ++i)
-        mbar_wait(&sh->v_full[i % v_stages], (i / v_stages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ntiles > 0) {
+    if (kQT && lane == 0 && ntiles > 0) {
+      // S_i = Q K_i^T with Q from TMEM, then O += P_i V_i, tile by tile: S_{i+1}
+      // overwrites S_i (and P_i) only after PV_i, which the tensor core runs
+      // in issue order; the other CTA on the SM fills the tensor core while this
+      // one's softmax works
+      const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
+      bool to = !mbar_wait(&sh->q_ready, 0, lim);
+      tc_fence_after();
+      for (int i = 0; i < ntiles && !to; ++i) {
+        const int s = i % k_stages;
+        if (!mbar_wait(&sh->k_full[s], (i / k_stages) & 1, lim)) {
+          to = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(k_ring + s * kTileBytes);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
+          mma_ts(tmem, tmem + 64 + k * 8, db, idesc_s, k > 0 ? 1u : 0u);
+        }
+        tc_commit(&sh->s_full[0][0]);
+        tc_commit(&sh->k_empty[s]);
+        if (!issue_pv(sh, v_ring, tmem, 1, i, v_stages, lim, true)) to = true;
+      }
+      if (to) atomicExch(&sh->timed_out, 1);
+      // Every MMA issued so far retires before TMEM and shared memory are
+      // released, also when a softmax warp gave up before reading the last O.
+      tc_commit(&sh->drain);
+      mbar_wait(&sh->drain, 0);
+    } else if (!kQT && lane == 0 && ntiles > 0) {
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
       bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
@@ -509,13 +599,35 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   float m = -INFINITY, l = 0.f;
   bool have = false;
   const bool warp_live = __any_sync(0xffffffffu, row_ok);  // some row of this warp is real
+  if (kQT && warp >= 2) {
+    // this thread's Q row (staged in shared memory before the allocation;
+    // zero for padding rows) -> TMEM columns [64, 128) of its lane, as bf16
+    // pairs: column j holds elements (2j, 2j+1), the A-operand layout
+    uint32_t qr[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v4 = *reinterpret_cast<const uint4*>(q_pipe + h * kRows * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+        qr[4 * c] = v4.x;
+        qr[4 * c + 1] = v4.y;
+        qr[4 * c + 2] = v4.z;
+        qr[4 * c + 3] = v4.w;
+      }
+      tmem_st32(t_s0 + lane_off + 64 + h * 32, qr);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh->q_ready);
+  }
   if (warp >= 2 && pipe < nq) {
     bool to = false;
     for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1;
+      const int sb = kQT ? 0 : (i & 1);
       // every wait that gates a TMEM access is decided for the whole warp: the
       // tcgen05.ld / tcgen05.st that follow are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[pipe][sb], (i >> 1) & 1, lim))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sh->s_full[pipe][sb], kQT ? (i & 1) : ((i >> 1) & 1), lim))) {
         to = true;
         break;
       }
@@ -685,7 +797,7 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
     // records per query tile (unit = (sequence, kv head, query tile)); chunk-major
     // ([32 float4 chunks][128 rows]) so that a warp's 32 rows write, and read
     // back, 512 contiguous bytes
-    const size_t n_units = (size_t)gridDim.z * tiles_q;
+    const size_t n_units = (size_t)p.B * p.Hkv * tiles_q;
     auto rec_o = [&](int qt) {
       return reinterpret_cast<float4*>(p.ws) + ((size_t)bh * tiles_q + qt) * ns * 32 * kRows;
     };
@@ -847,7 +959,7 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   p.v_stages = lp.v_stages;
   if ((int64_t)p.B * p.Hkv > 65535 || lp.tiles_q > 65535) return TV_ERR_UNSUPPORTED;
   const int grid_y = (lp.tiles_q + lp.nq - 1) / lp.nq;
-  dim3 grid(lp.nsplit, grid_y, p.B * p.Hkv);
+  dim3 grid(lp.nsplit, grid_y, p.B * p.Hkv);  // unit-major; query-tile-major below for one wave
   const int threads = 64 + 128 * lp.nq;
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
@@ -864,8 +976,9 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   int occ = 0;
   e = lp.nq == 2 ? occupancy(tree_attn_tc_kernel<2, false>, occ) : occupancy(tree_attn_tc_kernel<1, false>, occ);
   if (e != cudaSuccess) return record_cuda_error(e);
-  const bool lf = TV_TC_LONGEST_FIRST && lp.nq == 1 && p.B > 1 && p.B <= 32 &&
-                  (int64_t)grid.x * grid.y * grid.z > (int64_t)lp.per_sm * sms;
+  // multi-wave instance (unit-major, longest first) for one-tile CTAs whose grid
+  // exceeds the plan's resident CTAs; the single-wave instance otherwise
+  const bool lf = lp.nq == 1 && (int64_t)grid.x * grid.y * grid.z > (int64_t)lp.per_sm * sms;
   if (lf) {
     e = occupancy(tree_attn_tc_kernel<1, true>, occ);
     if (e != cudaSuccess) return record_cuda_error(e);
@@ -874,6 +987,7 @@ tv_status run_attention_tc(const CUtensorMap& tmk, const CUtensorMap& tmv, AttnP
   if (occ < 1 || occ * lp.nq > 2) return TV_ERR_UNSUPPORTED;
   auto kern = lp.nq == 2 ? tree_attn_tc_kernel<2, false>
                          : (lf ? tree_attn_tc_kernel<1, true> : tree_attn_tc_kernel<1, false>);
+  if (!lf && TV_TC_TILE_MAJOR) grid = dim3(lp.nsplit, p.B * p.Hkv, grid_y);
   return launch(kern, grid, dim3(threads), lp.smem, s, lp.nsplit, true, tmk, tmv, p);
 }
 
