@@ -87,6 +87,11 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_TILE_MAJOR
 #define TV_TC_TILE_MAJOR 1
 #endif
+//   TV_TC_MMA_POLL      1: the MMA thread polls its K, P and V barriers and
+//                       issues whichever MMA is ready (no head-of-line wait)
+#ifndef TV_TC_MMA_POLL
+#define TV_TC_MMA_POLL 1
+#endif
 //   TV_TC_SPLIT_PRODUCER 1: two producer threads, one per K and V stream
 #ifndef TV_TC_SPLIT_PRODUCER
 #define TV_TC_SPLIT_PRODUCER 1
@@ -239,6 +244,7 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   // Q in TMEM and one S buffer (one query tile per CTA): TMEM S [0,64),
   // Q [64,128), O [128,256); otherwise S0 [0,64), S1 [64,128), O [128,256)
   constexpr bool kQT = NQ == 1 && TV_TC_Q_TMEM;
+  constexpr bool kPoll = NQ == 1 && !kQT && TV_TC_MMA_POLL;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const bool aligned_ok = (smem_u32(smem_raw) & 1023u) == 0;
@@ -561,7 +567,68 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
       // released, also when a softmax warp gave up before reading the last O.
       tc_commit(&sh->drain);
       mbar_wait(&sh->drain, 0);
-    } else if (!kQT && lane == 0 && ntiles > 0) {
+    } else if (kPoll && lane == 0 && ntiles > 0) {
+      // One query tile, two S buffers.  QK_j may go once K_j has landed and
+      // PV_{j-2} is issued (it frees S[j % 2], which held P_{j-2}; the tensor
+      // core runs MMAs in issue order); PV_j once QK_j is issued and P_j and
+      // V_j are ready.  Polling both lets a late K tile hold back no PV and a
+      // late V tile no QK.  The wait limit applies to time without progress.
+      const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
+      const uint32_t idesc_o = idesc_bf16(128, 128, 1);
+      int nqk = 0, npv = 0;
+      bool to = false;
+      uint64_t t_last = globaltimer_ns();
+      uint32_t idle = 0;
+      while (npv < ntiles) {
+        bool progress = false;
+        if (nqk < ntiles && nqk < npv + 2 &&
+            mbar_test_wait(&sh->k_full[nqk % k_stages], (nqk / k_stages) & 1)) {
+          tc_fence_after();
+          const int s = nqk % k_stages, sb = nqk & 1;
+          const uint32_t k_addr = smem_u32(k_ring + s * kTileBytes);
+          const uint32_t q_addr = smem_u32(q_s);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
+            const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
+            mma_ss(tmem + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+          }
+          tc_commit(&sh->s_full[0][sb]);
+          tc_commit(&sh->k_empty[s]);
+          ++nqk;
+          progress = true;
+        }
+        if (npv < nqk && mbar_test_wait(&sh->p_full[0][npv & 1], (npv >> 1) & 1) &&
+            mbar_test_wait(&sh->v_full[npv % v_stages], (npv / v_stages) & 1)) {
+          tc_fence_after();
+          const int s = npv % v_stages, sb = npv & 1;
+          const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kKeyTile / 16; ++kk)
+            mma_ts(tmem + 128, tmem + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
+                   (npv > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&sh->o_ready[0][npv & 1]);
+          tc_commit(&sh->v_empty[s]);
+          ++npv;
+          progress = true;
+        }
+        if (progress) {
+          idle = 0;
+          t_last = globaltimer_ns();
+        } else if (++idle >= 64) {
+          idle = 0;
+          if (globaltimer_ns() - t_last > lim) {
+            to = true;
+            break;
+          }
+        }
+      }
+      if (to) atomicExch(&sh->timed_out, 1);
+      // Every MMA issued so far retires before TMEM and shared memory are
+      // released, also when a softmax warp gave up before reading the last O.
+      tc_commit(&sh->drain);
+      mbar_wait(&sh->drain, 0);
+    } else if (!kQT && !kPoll && lane == 0 && ntiles > 0) {
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
       bool to = false;
       for (int i = 0; i < ntiles && !to; ++i) {
