@@ -77,6 +77,33 @@ def test_parity_full(orc, B, M, Hq, Hkv, D, P):
     assert_attn_close(got, ref, f"B{B} M{M} Hq{Hq} Hkv{Hkv} D{D} P{P}")
 
 
+# Grids of more than one wave (320 CTAs of 2 query tiles on 148 SMs x 2): they
+# run the instance that starts (sequence, kv head) blocks longest prefix first.
+# B > 32 keeps row order; B = 1 ranks one row; the ragged batches put the
+# longest sequences in the middle and last, so the order moves rows around.
+@pytest.mark.parametrize("flags", [0, 1], ids=["plain", "prefix_ready"])
+@pytest.mark.parametrize(
+    "B,M,Hq,Hkv,P,left",
+    [
+        (40, 16, 32, 4, "ragged", False),  # more rows than one warp ranks: row order
+        (1, 130, 160, 160, [100], False),  # one sequence, many heads
+        (20, 40, 32, 8, "ragged", True),  # longest first changes which row each block serves
+    ],
+    ids=["B40", "B1", "B20_left_padded"],
+)
+def test_multi_wave_block_order(orc, B, M, Hq, Hkv, P, left, flags):
+    if P == "ragged":
+        rng = np.random.default_rng(B)
+        P = rng.integers(16, 300, size=B).astype(np.int32)
+        P[B // 2] = 500  # the longest in the middle ...
+        P[-1] = 499  # ... and the second longest last
+    q, k, v, par, ks, kl = _inputs(B, M, Hq, Hkv, 128, P, seed=7000 + B, left_padded=left)
+    got, ref, status = _run(orc, q, k, v, par, ks, kl, flags=flags)
+    assert not status.any().item()
+    assert not np.isnan(got).any()
+    assert_attn_close(got, ref, f"multi-wave B{B} M{M} Hq{Hq} Hkv{Hkv} flags{flags}")
+
+
 def test_left_padded_ragged(orc):
     q, k, v, par, ks, kl = _inputs(5, 7, 16, 4, 128, [10, 700, 64, 1, 1500], seed=3, left_padded=True)
     got, ref, _ = _run(orc, q, k, v, par, ks, kl)
