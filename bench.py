@@ -390,7 +390,7 @@ def build_workload(cfg, seed, device, L_phys=None, extra_rows=0):
 def per_call_times(ver, cfg, stream, reps, reset):
     """Device time (ms) of each call alone: graphs, inputs resident."""
     L = cfg.L
-    g_attn = capture(lambda: [ver.attention(layer, stream, prefix_ready=True) for layer in range(L)], stream)
+    g_attn = capture(lambda: [ver.attention(layer, stream) for layer in range(L)], stream)
     with torch.cuda.stream(stream):
         for _ in range(3):
             g_attn.replay()
@@ -415,7 +415,7 @@ def per_call_times(ver, cfg, stream, reps, reset):
     ver.rope_theta = 10000.0
     attn_rope_ms = None
     if cfg.D == 128:  # the rotation is fused into the head dim 128 kernel only
-        g_r = capture(lambda: [ver.attention(layer, stream, prefix_ready=True) for layer in range(L)], stream)
+        g_r = capture(lambda: [ver.attention(layer, stream) for layer in range(L)], stream)
         attn_rope_ms = event_time(g_r.replay, reps, stream) / L
         del g_r
     g_w = capture(lambda: [ver.write_tree_rows(layer, stream) for layer in range(L)], stream)
@@ -735,7 +735,7 @@ def measure_rounds(args, cfg, world, device, rounds, replays, warmup, with_clock
             tv.tree_kv_write(ver.k_ptrs[layer:layer + 1], ver.v_ptrs[layer:layer + 1], tk_r[r, layer:layer + 1],
                              tv_r[r, layer:layer + 1], ver.S_cap, ver.kv_start, ver.kv_len, stream)
             tv.tree_attention(q_r[r, layer], ver.k[layer], ver.v[layer], ver.kv_start, ver.kv_len, ver.anc,
-                              ver.status, ver.out[layer], ver.workspace, stream=stream, flags=tv.ATTN_PREFIX_READY)
+                              ver.status, ver.out[layer], ver.workspace, stream=stream)
         tv.tree_accept(lg_r[r], dr_r[r], ver.parent, ver.depth, ver.anc, ver.status, cfg.max_depth, am, al_r[r],
                        path_r[r], bonus_r[r], stream)
         tv.kv_commit_realign(ver.k_commit_ptrs, ver.v_commit_ptrs, B, cfg.Hkv, cfg.D, ver.S_cap, cfg.M, path_r[r],
@@ -808,7 +808,7 @@ def measure_rounds(args, cfg, world, device, rounds, replays, warmup, with_clock
     def attn_round0():
         for layer in range(L):
             tv.tree_attention(q_r[0, layer], ver.k[layer], ver.v[layer], ver.kv_start, ver.kv_len, ver.anc,
-                              ver.status, ver.out[layer], ver.workspace, stream=stream, flags=tv.ATTN_PREFIX_READY)
+                              ver.status, ver.out[layer], ver.workspace, stream=stream)
 
     g_a = capture(attn_round0, stream)
     with torch.cuda.stream(stream):
@@ -1278,7 +1278,7 @@ def run_profile(args, cfg):
         ver.build_mask(stream)
         for _ in range(3):
             if args.profile == "attention":
-                ver.attention(0, stream, prefix_ready=True)
+                ver.attention(0, stream)
             else:
                 ver.kv_start.copy_(torch.as_tensor(host["kv_start"], device=device))
                 ver.kv_len.copy_(torch.as_tensor(host["kv_len"], device=device))

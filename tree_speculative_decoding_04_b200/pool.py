@@ -163,8 +163,7 @@ class PoolVerifier:
                              self.tree_k[layer:layer + 1, :Bb], self.tree_v[layer:layer + 1, :Bb], self.S_cap,
                              self.kv_start, self.kv_len, s, slot=sl)
             tv.tree_attention(self.q[layer, :Bb], self.k[layer], self.v[layer], self.kv_start, self.kv_len,
-                              self.anc[:Bb], self.status[:Bb], self.out[layer, :Bb], self._ws(Bb), stream=s,
-                              flags=tv.ATTN_PREFIX_READY, slot=sl)  # follows tree_kv_write
+                              self.anc[:Bb], self.status[:Bb], self.out[layer, :Bb], self._ws(Bb), stream=s, slot=sl)
         tv.tree_accept(self.logits[:Bb], self.draft[:Bb], self.parent[:Bb], self.depth[:Bb], self.anc[:Bb],
                        self.status[:Bb], self.max_depth, self.argmax[:Bb], self.accept_len[:Bb], self.path[:Bb],
                        self.bonus[:Bb], s)
