@@ -254,7 +254,11 @@ def realign_geometry(kv_start, kv_len, accept_len, realign):
 # ----------------------------------------------------------------------------- timing helpers
 
 def event_time(fn, reps, stream):
-    """Mean device time (ms) of fn(), launched on `stream`, over reps back-to-back calls."""
+    """Mean device time (ms) of fn(), launched on `stream`, over reps back-to-back
+    calls, after one untimed call (the first replay of a captured graph also
+    uploads it)."""
+    with torch.cuda.stream(stream):
+        fn()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
