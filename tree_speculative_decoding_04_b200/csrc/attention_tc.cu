@@ -72,6 +72,15 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_V_RING_SOLO
 #define TV_TC_V_RING_SOLO 6
 #endif
+// ring depths (K, V) of a CTA that shares its SM with another (up to 5 slots
+// fit; 2 + 2 measured faster than 2 + 3 and 3 + 2 on B200: mha7b 17.6 vs
+// 18.4 us, b32gqa 151 vs 154 us, stress the same)
+#ifndef TV_TC_K_RING_DUO
+#define TV_TC_K_RING_DUO 2
+#endif
+#ifndef TV_TC_V_RING_DUO
+#define TV_TC_V_RING_DUO 2
+#endif
 //   TV_TC_LONGEST_FIRST  1: grids of more than one wave start their (sequence,
 //                       kv head) blocks longest prefix first
 #ifndef TV_TC_LONGEST_FIRST
@@ -1007,10 +1016,11 @@ tv_status plan_attention_tc(int B, int M, int Hq, int Hkv, int64_t S_cap, TcPlan
     const int64_t ctas = ctas_per_split * lp.nsplit;
     const bool two_per_sm = !TV_TC_FORCE_SOLO && (!TV_TC_ONE_PER_SM || ctas > sms);
     lp.per_sm = two_per_sm ? 2 : 1;
-    // two CTAs per SM: K ring 2, V ring 3 (Q 32 KB + 5 x 16 KB fits twice in an SM);
+    // two CTAs per SM: K and V rings of TV_TC_K_RING_DUO / TV_TC_V_RING_DUO slots
+    // (Q 32 KB + up to 5 x 16 KB fits twice in an SM);
     // one CTA per SM: deeper rings
-    lp.stages = two_per_sm ? 2 : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
-    lp.v_stages = two_per_sm ? 3 : std::min(TV_TC_V_RING_SOLO, std::max(2, lp.tiles_per_split));
+    lp.stages = two_per_sm ? TV_TC_K_RING_DUO : std::min(TV_TC_K_RING_SOLO, std::max(2, lp.tiles_per_split));
+    lp.v_stages = two_per_sm ? TV_TC_V_RING_DUO : std::min(TV_TC_V_RING_SOLO, std::max(2, lp.tiles_per_split));
     const size_t smem_min = two_per_sm ? 0 : (size_t)120 * 1024;  // > half the SM: one CTA per SM
     lp.smem = std::max(smem_min, kQBytes + (size_t)(lp.stages + lp.v_stages) * kTileBytes + sizeof(TcSmem));
   }
