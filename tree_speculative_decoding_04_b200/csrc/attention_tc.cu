@@ -72,6 +72,17 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_V_RING_SOLO
 #define TV_TC_V_RING_SOLO 6
 #endif
+//   TV_TC_PREFETCH_TILES key tiles per CTA warmed in L2 before the grid dependency
+//                       (0: measured fastest on B200, the early requests
+//                       compete with the launch still running)
+//   TV_TC_PREFETCH_Q     1: the CTA's query rows are warmed in L2 before it
+//                       (0: measured as fast or faster)
+#ifndef TV_TC_PREFETCH_TILES
+#define TV_TC_PREFETCH_TILES 0
+#endif
+#ifndef TV_TC_PREFETCH_Q
+#define TV_TC_PREFETCH_Q 0
+#endif
 // ring depths (K, V) of a CTA that shares its SM with another (up to 5 slots
 // fit; 2 + 2 measured faster than 2 + 3 and 3 + 2 on B200: mha7b 17.6 vs
 // 18.4 us, b32gqa 151 vs 154 us, stress the same)
@@ -115,7 +126,7 @@ constexpr int kMaxStages = 8;
 constexpr int kQBytes = kRows * 128 * 2;         // 2 boxes of [128 rows][128 B]
 constexpr int kTileBytes = kKeyTile * 128 * 2;   // K (or V): 2 boxes of [64 rows][128 B]
 constexpr float kRescaleThreshold = 8.0f;        // log2 domain
-constexpr int kPrefetchTiles = 1;                 // key tiles per CTA warmed in L2 before the grid dependency
+constexpr int kPrefetchTiles = TV_TC_PREFETCH_TILES;  // key tiles per CTA warmed in L2 before the grid dependency
 constexpr int kMaxSplit_tc = 8;                  // portable cluster size
 
 struct TcSmem {
@@ -351,11 +362,12 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   // limit of the pipeline waits; the waits that drain copies or MMAs in flight
   // before the CTA exits always keep the full limit
   const uint64_t lim = p.wait_limit_ns;
-  // Warp 0 reads the row order and the geometry before the grid dependency
-  // (one round trip); the other warps read them after it only.
+  // With TV_ATTN_PREFIX_READY (or key tiles to warm in L2), warp 0 reads the
+  // row order and the geometry before the grid dependency (one round trip);
+  // otherwise every warp reads them after it only.
   RowGeo pre{rank, -1, 0, 0, 0, 0};
   int npre_k = 0, npre_v = 0;  // tiles requested before the grid dependency
-  if (warp == 0) {
+  if (warp == 0 && (prefix_ready || kPrefetchTiles > 0)) {
     pre = row_of_rank<LF>(p, rank);
     if (prefix_ready) {
       if (pre.sl >= 0 && aligned_ok && geometry_ok(pre.ks, pre.kl, p.M, p.S_cap)) {
@@ -389,7 +401,7 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
     }
   }
   // the query rows are warmed in L2 when the row is known without a load
-  if (warp >= 2 && (!LF || p.B > 32)) {
+  if (TV_TC_PREFETCH_Q && warp >= 2 && (!LF || p.B > 32)) {
     const int gr_h = (qtile0 + ((warp - 2) >> 2)) * kRows + (warp & 3) * 32 + lane;
     if (gr_h < p.rows_total) {
       const uint16_t* qr =
