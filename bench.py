@@ -965,9 +965,12 @@ def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
         pv.draft[:Bb].copy_(drafts[r % rounds][:Bb])
         pv.set_slots(slots, stream)
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        realign = 1 if mode == FALLBACK else 0
+        pv.graphs(Bb, realign, stream)  # captured on first use, before the timed region
+        stream.wait_stream(torch.cuda.current_stream(device))  # this round's logits and drafts
         with torch.cuda.stream(stream):
             e0.record(stream)
-            pv.step(Bb, 1 if mode == FALLBACK else 0, stream, before_commit=lambda: e1.record(stream))
+            pv.step_graphed(Bb, realign, stream, between=lambda: e1.record(stream))
             e2.record(stream)
         e2.synchronize()
         al = pv.accept_len[:Bb].cpu().numpy()
@@ -992,7 +995,8 @@ def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
         "commit_ms_per_round": {k: v / max(1, n_grouped if k == "grouped" else n_fallback)
                                 for k, v in com_by_mode.items()},
         "gpu_launches_per_round": pv.launches_per_step(),
-        "note": "every round ends with a host synchronisation (the scheduler needs the accept lengths)",
+        "note": "each round replays the step's CUDA graphs (captured once per batch size and mode) with its slot "
+                "map; every round ends with a host synchronisation (the scheduler needs the accept lengths)",
     }
     del pv, lg, drafts
     return rec

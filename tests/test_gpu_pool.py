@@ -19,8 +19,11 @@ from tree_speculative_decoding_04_b200.pool import FALLBACK, PoolVerifier, Seque
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("graphed", [False, True], ids=["eager", "graphs"])
 @pytest.mark.parametrize("tree", ["uniform_depth", "chain"])
-def test_pool_rounds_against_the_oracle(orc, tree):
+def test_pool_rounds_against_the_oracle(orc, tree, graphed):
+    """Eager launches, or the step's CUDA graphs captured once per (batch size,
+    mode) and replayed with each round's slot map."""
     rng = np.random.default_rng(3 if tree == "chain" else 4)
     g = W.torch_generator(5, dev())
     n_slots, B, L, Hq, Hkv, D, M, max_depth, V = 10, 4, 2, 8, 2, 128, 5, 5, 2048
@@ -39,6 +42,7 @@ def test_pool_rounds_against_the_oracle(orc, tree):
     mask_h = np.zeros((n_slots, S_cap), np.uint8)
     pos_h = np.zeros((n_slots, S_cap), np.int32)
     pool = SequencePool(lengths0, batch=B, max_wait=4)
+    side = torch.cuda.Stream(dev())
     modes = set()
     for rnd in range(rounds):
         slots, mode = pool.next_batch()
@@ -56,8 +60,13 @@ def test_pool_rounds_against_the_oracle(orc, tree):
         pv.tree_k[:, :Bb].copy_(W.randn_bf16((L, Bb, Hkv, M + 1, D), g, dev()))
         pv.tree_v[:, :Bb].copy_(W.randn_bf16((L, Bb, Hkv, M + 1, D), g, dev()))
         realign = 1 if mode == FALLBACK else 0
-        pv.set_slots(slots)
-        pv.step(Bb, realign)
+        if graphed:
+            torch.cuda.synchronize()  # the inputs above are on the default stream
+            pv.set_slots(slots, side)
+            pv.step_graphed(Bb, realign, side)
+        else:
+            pv.set_slots(slots)
+            pv.step(Bb, realign)
         torch.cuda.synchronize()
         # the oracle on the same inputs
         anc, depth, st = orc.tree_build_mask(parent, max_depth)

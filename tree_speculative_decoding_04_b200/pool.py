@@ -132,6 +132,7 @@ class PoolVerifier:
         self.path = torch.zeros((B, max_depth + 1), **i32)
         self.bonus = torch.zeros((B,), **i32)
         self.workspace = {}
+        self._graphs = {}
 
     def _ws(self, Bb):
         if Bb not in self.workspace:
@@ -156,6 +157,13 @@ class PoolVerifier:
         run (on the host) between the accept and the commit launches, e.g. to
         record a CUDA event."""
         s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self._step_main(Bb, s)
+        if before_commit is not None:
+            before_commit()
+        self._step_commit(Bb, realign, s)
+
+    def _step_main(self, Bb, s):
+        """mask, per layer tree_kv_write + attention, accept"""
         sl = self.slot[:Bb]
         tv.tree_build_mask(self.parent[:Bb], self.max_depth, self.anc[:Bb], self.depth[:Bb], self.status[:Bb], s)
         for layer in range(self.L):
@@ -167,11 +175,43 @@ class PoolVerifier:
         tv.tree_accept(self.logits[:Bb], self.draft[:Bb], self.parent[:Bb], self.depth[:Bb], self.anc[:Bb],
                        self.status[:Bb], self.max_depth, self.argmax[:Bb], self.accept_len[:Bb], self.path[:Bb],
                        self.bonus[:Bb], s)
-        if before_commit is not None:
-            before_commit()
+
+    def _step_commit(self, Bb, realign, s):
+        sl = self.slot[:Bb]
         tv.kv_commit_realign(self.k_ptrs, self.v_ptrs, Bb, self.Hkv, self.D, self.S_cap, self.M, self.path[:Bb],
                              self.accept_len[:Bb], self.status[:Bb], self.max_depth, self.kv_start, self.kv_len,
                              self.max_len, int(realign), self.attn_mask, self.pos_ids, s, slot=sl)
+
+    def graphs(self, Bb, realign, stream):
+        """CUDA graphs of one step of the first Bb batch rows, captured once per
+        (Bb, realign) and replayed: (everything up to the accept, the commit).
+        The slot map and the per-slot geometry are read on the device, so one
+        pair of graphs serves every batch of that size and mode; set_slots
+        before each replay."""
+        key = (int(Bb), int(realign))
+        if key not in self._graphs:
+            s = stream
+            self._ws(Bb)  # allocated outside the capture
+            g_main, g_commit = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            # two graphs: the launches before the commit, then the commit
+            with torch.cuda.graph(g_main, stream=s):
+                self._step_main(Bb, s)
+            with torch.cuda.graph(g_commit, stream=s):
+                self._step_commit(Bb, realign, s)
+            self._graphs[key] = (g_main, g_commit)
+        return self._graphs[key]
+
+    def step_graphed(self, Bb, realign, stream=None, between=None):
+        """step() through the captured graphs (asynchronous on `stream`, which
+        must be a side stream, not the default one); between: optional callable
+        run on the host between the two replays, e.g. to record a CUDA event."""
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        g_main, g_commit = self.graphs(Bb, realign, s)
+        with torch.cuda.stream(s):
+            g_main.replay()
+            if between is not None:
+                between()
+            g_commit.replay()
 
     def launches_per_step(self) -> int:
         """mask 1, per layer tree_kv_write 1 + attention 1, accept 2, commit 2."""
