@@ -918,7 +918,7 @@ def measure_lm_head(args, cfg, device, reps=5):
                     "widened to fp32, then tree_accept"}
 
 
-def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
+def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4, repad=True):
     """Cross-batch scheduling (EXSPEC) on the EQSPEC shapes: a pool of n_slots
     sequences whose prefix lengths come from a few length buckets (drawn from the
     workload's range), batches of up to B picked every round by SequencePool
@@ -965,7 +965,7 @@ def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
         pv.draft[:Bb].copy_(drafts[r % rounds][:Bb])
         pv.set_slots(slots, stream)
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        realign = 1 if mode == FALLBACK else 0
+        realign = 1 if (mode == FALLBACK and repad) else 0
         pv.graphs(Bb, realign, stream)  # captured on first use, before the timed region
         stream.wait_stream(torch.cuda.current_stream(device))  # this round's logits and drafts
         with torch.cuda.stream(stream):
@@ -994,6 +994,8 @@ def measure_exspec(args, cfg, device, rounds=64, n_slots=32, buckets=4):
         "commit_share_of_device_time": com_ms / dev_ms,
         "commit_ms_per_round": {k: v / max(1, n_grouped if k == "grouped" else n_fallback)
                                 for k, v in com_by_mode.items()},
+        "fallback_commit": "EQSPEC repad (the pages' EXSPEC)" if repad else
+                           "per sequence, no repad (the slot map's per-sequence geometry; beyond the pages)",
         "gpu_launches_per_round": pv.launches_per_step(),
         "note": "each round replays the step's CUDA graphs (captured once per batch size and mode) with its slot "
                 "map; every round ends with a host synchronisation (the scheduler needs the accept lengths)",
@@ -1209,6 +1211,10 @@ def run_ours(args, cfg, world, rank, local):
                     eq["kv_commit"]["us"] * 1e-3 / eq["ms_per_round"])
         except Exception as e:
             per_config["exspec"] = {"error": repr(e)[:300]}
+        try:
+            per_config["exspec_ragged_fallback"] = measure_exspec(args, W.CONFIGS["eqspec"], device, repad=False)
+        except Exception as e:
+            per_config["exspec_ragged_fallback"] = {"error": repr(e)[:300]}
         free_state({})
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

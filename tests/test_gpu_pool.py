@@ -19,11 +19,16 @@ from tree_speculative_decoding_04_b200.pool import FALLBACK, PoolVerifier, Seque
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("graphed", [False, True], ids=["eager", "graphs"])
-@pytest.mark.parametrize("tree", ["uniform_depth", "chain"])
-def test_pool_rounds_against_the_oracle(orc, tree, graphed):
+@pytest.mark.parametrize(
+    "tree,graphed,repad",
+    [("uniform_depth", False, True), ("chain", False, True), ("uniform_depth", True, True), ("chain", True, True),
+     ("uniform_depth", True, False)],
+    ids=["uniform_depth-eager", "chain-eager", "uniform_depth-graphs", "chain-graphs", "ragged_fallback-graphs"])
+def test_pool_rounds_against_the_oracle(orc, tree, graphed, repad):
     """Eager launches, or the step's CUDA graphs captured once per (batch size,
-    mode) and replayed with each round's slot map."""
+    mode) and replayed with each round's slot map.  repad: fallback batches take
+    the EQSPEC repad (the pages' EXSPEC); else they commit per sequence like
+    grouped ones (the slot map's per-sequence geometry needs no alignment)."""
     rng = np.random.default_rng(3 if tree == "chain" else 4)
     g = W.torch_generator(5, dev())
     n_slots, B, L, Hq, Hkv, D, M, max_depth, V = 10, 4, 2, 8, 2, 128, 5, 5, 2048
@@ -59,7 +64,7 @@ def test_pool_rounds_against_the_oracle(orc, tree, graphed):
         pv.q[:, :Bb].copy_(W.randn_bf16((L, Bb, M + 1, Hq, D), g, dev()))
         pv.tree_k[:, :Bb].copy_(W.randn_bf16((L, Bb, Hkv, M + 1, D), g, dev()))
         pv.tree_v[:, :Bb].copy_(W.randn_bf16((L, Bb, Hkv, M + 1, D), g, dev()))
-        realign = 1 if mode == FALLBACK else 0
+        realign = 1 if (mode == FALLBACK and repad) else 0
         if graphed:
             torch.cuda.synchronize()  # the inputs above are on the default stream
             pv.set_slots(slots, side)
