@@ -28,8 +28,9 @@ def load_golden(name):
 
 # Raw error statistics of every attention comparison of the session, by label:
 # max |gpu - ref| over all elements, and max |gpu - ref| / |ref| over the
-# elements with |ref| >= 0.1 (the benchmark spec's max-abs / max-rel figures, which
-# the allclose bar above combines).  Printed at the end of the session.
+# elements with |ref| >= 0.1 (the max-abs 1e-2 / max-rel 2e-2 figures of the
+# attention tolerance, which the allclose bar above combines).  Printed at the
+# end of the session.
 ERR_STATS = {}
 
 
