@@ -116,6 +116,17 @@ namespace cg = cooperative_groups;
 #ifndef TV_TC_SPLIT_PRODUCER
 #define TV_TC_SPLIT_PRODUCER 1
 #endif
+//   TV_TC_EARLY_ROWS    1: grids in row order request the query rows before
+//                       the geometry
+#ifndef TV_TC_EARLY_ROWS
+#define TV_TC_EARLY_ROWS 1
+#endif
+//   TV_TC_DESC_STEP     1: the polling MMA thread forms each k-step's
+//                       shared-memory descriptor as the tile's first one plus a
+//                       constant (one add per MMA)
+#ifndef TV_TC_DESC_STEP
+#define TV_TC_DESC_STEP 1
+#endif
 
 namespace tv {
 namespace {
@@ -419,6 +430,34 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
   // flagged instead of computed; a changed length may also have changed the
   // row order, which CTAs that read early no longer share with the others, so
   // then every row of the batch is flagged.
+  const int pipe = warp >= 2 ? (warp - 2) >> 2 : 0;  // query pipe of a softmax warp
+  const int qtile = qtile0 + pipe;
+  uint8_t* q_pipe = q_s + pipe * kQBytes;
+  const uint32_t tq = (uint32_t)(pipe * kTmemCols);  // column offset of this pipe's TMEM block
+  const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
+  const int gr = qtile * kRows + r;
+  const bool row_ok = pipe < nq && gr < p.rows_total;
+  const int hq = hk * p.G + gr % p.G;
+  const int u = min(gr / p.G, p.M);
+  // A softmax thread's query row (zero past the tile), its ancestor words and,
+  // with TV_ATTN_ROPE, its tree depth.  A grid in row order serves batch row
+  // `rank`, known without a load, so these requests go out before the
+  // geometry's and the two round trips overlap; the longest-first instance
+  // learns its row from the geometry and requests them after it.
+  constexpr bool kEarlyRows = !LF && TV_TC_EARLY_ROWS;
+  uint4 qv[16];
+  uint32_t anc_w[kMaxRows / 32];
+  int depth_u = 0;
+  auto load_rows = [&](int b_) {
+    const int64_t node = (int64_t)b_ * (p.M + 1) + u;
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + (node * p.Hq + hq) * 128);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) qv[c] = row_ok ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    if ((p.flags & TV_ATTN_ROPE) && row_ok) depth_u = p.depth[node];
+#pragma unroll
+    for (int w = 0; w < kMaxRows / 32; ++w) anc_w[w] = w < p.W ? __ldg(p.anc + node * p.W + w) : 0u;
+  };
+  if (kEarlyRows && warp >= 2) load_rows(rank);
   const RowGeo g = row_of_rank<LF>(p, rank);
   const int b = g.b;
   const int sl = g.sl;
@@ -449,38 +488,21 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
       if (lane == 0 && i < k_stages && i >= npre_k) issue_k(i, ks, k_lo, zc);
       if (lane == (TV_TC_SPLIT_PRODUCER ? 1 : 0) && i < v_stages && i >= npre_v) issue_v(i, ks, k_lo, zc);
     }
-  const int pipe = warp >= 2 ? (warp - 2) >> 2 : 0;  // query pipe of a softmax warp
-  const int qtile = qtile0 + pipe;
-  uint8_t* q_pipe = q_s + pipe * kQBytes;
-  const uint32_t tq = (uint32_t)(pipe * kTmemCols);  // column offset of this pipe's TMEM block
-  const int r = (warp & 3) * 32 + lane;  // TMEM lane == query row of this tile
-  const int gr = qtile * kRows + r;
-  const bool row_ok = pipe < nq && gr < p.rows_total;
-  const int hq = hk * p.G + gr % p.G;
-  const int u = min(gr / p.G, p.M);
-  uint32_t anc_w[kMaxRows / 32];
   if (warp >= 2) {
+    if (!kEarlyRows) load_rows(b);
     // Q row -> swizzled smem (two 64-column boxes); rows past the tile are zero.
     // With TV_ATTN_ROPE the row is rotated to its tree position kv_len +
     // depth(u) on the way (pairs (i, i + 64) sit in chunks c and c + 8).
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * (p.M + 1) + u) * p.Hq + hq) * 128);
     const bool rope = (p.flags & TV_ATTN_ROPE) != 0;
-    const int pos = (rope && row_ok) ? kl + p.depth[(int64_t)b * (p.M + 1) + u] : 0;
+    const int pos = (rope && row_ok) ? kl + depth_u : 0;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-      if (row_ok) {
-        lo = __ldg(src + c);
-        hi = __ldg(src + c + 8);
-        if (rope) rope_rotate8(lo, hi, pos, p.rope.f, 8 * c);
-      }
+      uint4 lo = qv[c], hi = qv[c + 8];
+      if (row_ok && rope) rope_rotate8(lo, hi, pos, p.rope.f, 8 * c);
       *reinterpret_cast<uint4*>(q_pipe + r * 128 + ((c ^ (r & 7)) << 4)) = lo;
       *reinterpret_cast<uint4*>(q_pipe + kRows * 128 + r * 128 + ((c ^ (r & 7)) << 4)) = hi;
     }
     fence_async_smem();  // generic-proxy stores -> visible to the tensor core after the barrier
-#pragma unroll
-    for (int w = 0; w < kMaxRows / 32; ++w)
-      anc_w[w] = w < p.W ? __ldg(p.anc + ((int64_t)b * (p.M + 1) + u) * p.W + w) : 0u;
   }
   if (warp == 1) {
     __syncwarp();  // tcgen05.alloc is warp-collective
@@ -596,6 +618,8 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
       // late V tile no QK.  The wait limit applies to time without progress.
       const uint32_t idesc_s = idesc_bf16(128, kKeyTile, 0);
       const uint32_t idesc_o = idesc_bf16(128, 128, 1);
+      constexpr bool kDescStep = TV_TC_DESC_STEP != 0;
+      const uint64_t dq0 = sw128_desc(smem_u32(q_s), 16);  // the query tile's first k-step
       int nqk = 0, npv = 0;
       bool to = false;
       uint64_t t_last = globaltimer_ns();
@@ -607,12 +631,24 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
           tc_fence_after();
           const int s = nqk % k_stages, sb = nqk & 1;
           const uint32_t k_addr = smem_u32(k_ring + s * kTileBytes);
-          const uint32_t q_addr = smem_u32(q_s);
+          if (kDescStep) {
+            // the k-steps' descriptors differ from the tile's first one only in
+            // the address field (16-byte units, bits 0-13; every address stays
+            // below 256 KB, so the sum never carries out of the field): one add
+            // per MMA keeps the issuing thread's dependent chain short
+            const uint64_t dk0 = sw128_desc(k_addr, 16);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
-            const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
-            mma_ss(tmem + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+            for (int k = 0; k < 8; ++k)
+              mma_ss(tmem + sb * 64, dq0 + (uint64_t)((k >> 2) * (kRows * 128 / 16) + (k & 3) * 2),
+                     dk0 + (uint64_t)((k >> 2) * (kBoxBytes / 16) + (k & 3) * 2), idesc_s, k > 0 ? 1u : 0u);
+          } else {
+            const uint32_t q_addr = smem_u32(q_s);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint64_t da = sw128_desc(q_addr + (k >> 2) * (kRows * 128) + (k & 3) * 32, 16);
+              const uint64_t db = sw128_desc(k_addr + (k >> 2) * kBoxBytes + (k & 3) * 32, 16);
+              mma_ss(tmem + sb * 64, da, db, idesc_s, k > 0 ? 1u : 0u);
+            }
           }
           tc_commit(&sh->s_full[0][sb]);
           tc_commit(&sh->k_empty[s]);
@@ -624,10 +660,18 @@ __global__ void __launch_bounds__(64 + 128 * NQ, NQ == 1 ? 2 : 1)
           tc_fence_after();
           const int s = npv % v_stages, sb = npv & 1;
           const uint32_t v_addr = smem_u32(v_ring + s * kTileBytes);
+          if (kDescStep) {
+            const uint64_t dv0 = sw128_desc(v_addr, kBoxBytes);
 #pragma unroll
-          for (int kk = 0; kk < kKeyTile / 16; ++kk)
-            mma_ts(tmem + 128, tmem + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
-                   (npv > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kKeyTile / 16; ++kk)
+              mma_ts(tmem + 128, tmem + sb * 64 + kk * 8, dv0 + (uint64_t)(kk * (16 * 128 / 16)), idesc_o,
+                     (npv > 0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kKeyTile / 16; ++kk)
+              mma_ts(tmem + 128, tmem + sb * 64 + kk * 8, sw128_desc(v_addr + kk * 16 * 128, kBoxBytes), idesc_o,
+                     (npv > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit(&sh->o_ready[0][npv & 1]);
           tc_commit(&sh->v_empty[s]);
           ++npv;
