@@ -8,15 +8,16 @@
 // tensor memory and reduced to (max, first index) on the spot, so the
 // [rows][V] logits never reach HBM.
 //
-// Design (one CTA per output tile of 128 rows x 256 vocabulary columns; rows =
-// B * (M+1) tree nodes, H the hidden size):
+// Design (one CTA per output tile of 128 rows x bn vocabulary columns, bn = 256
+// or, for grids of a few waves, the multiple of 32 that fills the SMs best;
+// rows = B * (M+1) tree nodes, H the hidden size):
 //   warp 0      TMA producer: per 64-wide K slab, the hidden tile (128 x 64,
-//               16 KB) and the weight tile (256 x 64, 32 KB), both K-major with
-//               the 128-byte swizzle, into a 4-stage ring
+//               16 KB) and the weight tile (bn x 64, up to 32 KB), both K-major
+//               with the 128-byte swizzle, into a 4-stage ring
 //   warp 1      TMEM owner (256 columns) and MMA issuer: 4 x tcgen05.mma
-//               (M=128, N=256, K=16) per slab, fp32 accumulation in TMEM
+//               (M=128, N=bn, K=16) per slab, fp32 accumulation in TMEM
 //   warps 2-5   epilogue: thread t owns TMEM lane t (= tile row t); it reads its
-//               256 logits 32 at a time and keeps the first maximum, then merges
+//               bn logits 32 at a time and keeps the first maximum, then merges
 //               (max, index) into the row's 64-bit key with one atomicMax: the
 //               key orders by value first and by lower index second, so the
 //               merge over the vocabulary tiles keeps the first maximum.
@@ -32,7 +33,7 @@ namespace {
 
 constexpr int kLmThreads = 192;
 constexpr int kBM = 128;  // rows per tile (TMEM lanes)
-constexpr int kBN = 256;  // vocabulary columns per tile (TMEM columns)
+constexpr int kBN = 256;  // most vocabulary columns per tile (TMEM columns)
 constexpr int kBK = 64;   // K slab: 128 bytes of bf16, one swizzle row
 constexpr int kLmStages = 4;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB
@@ -63,14 +64,15 @@ __global__ void __launch_bounds__(kLmThreads) lm_keys_init_kernel(unsigned long 
 
 __global__ void __launch_bounds__(kLmThreads, 1) lm_head_argmax_kernel(
     const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b, int rows, int H, int V,
-    int m_tiles, int node_rows, unsigned long long* __restrict__ keys, int32_t* __restrict__ status, uint64_t lim) {
+    int m_tiles, int bn, int node_rows, unsigned long long* __restrict__ keys, int32_t* __restrict__ status,
+    uint64_t lim) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const bool aligned_ok = (smem_u32(smem) & 1023u) == 0;
   LmSmem* sh = reinterpret_cast<LmSmem*>(smem + kLmStages * kLmStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x;
   const int row0 = (tile % m_tiles) * kBM;
-  const int col0 = (tile / m_tiles) * kBN;
+  const int col0 = (tile / m_tiles) * bn;
   const int nk = H / kBK;
 
   if (threadIdx.x == 0) {
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lm_head_argmax_kernel(
           break;
         }
         uint8_t* a = smem + s * kLmStageBytes;
-        mbar_arrive_expect_tx(&sh->full[s], kLmStageBytes);
+        mbar_arrive_expect_tx(&sh->full[s], kABytes + bn * kBK * 2);
         tma_load_2d(a, &tma_a, &sh->full[s], kt * kBK, row0);
         tma_load_2d(a + kABytes, &tma_b, &sh->full[s], kt * kBK, col0);
         ++issued;
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lm_head_argmax_kernel(
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && run) {
-      const uint32_t idesc = idesc_bf16(kBM, kBN, 0);
+      const uint32_t idesc = idesc_bf16(kBM, bn, 0);
       bool to = false;
       for (int kt = 0; kt < nk; ++kt) {
         const int s = kt % kLmStages;
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(kLmThreads, 1) lm_head_argmax_kernel(
       float best = -INFINITY;
       int bi = -1;
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < bn / 32; ++c) {
         uint32_t x[32];
         tmem_ld32(tmem + lane_off + c * 32, x);
         tmem_wait_ld();
@@ -243,17 +245,34 @@ extern "C" tv_status tree_accept_lm_head(const uint16_t* hidden, const uint16_t*
   const int64_t rows = (int64_t)B * (M + 1);
   if (workspace_bytes < (size_t)rows * sizeof(unsigned long long)) return TV_ERR_INVALID_ARG;
   const int m_tiles = (int)((rows + kBM - 1) / kBM);
-  const int64_t n_tiles = ((int64_t)V + kBN - 1) / kBN;
-  if ((int64_t)m_tiles * n_tiles > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
-  CUtensorMap ta, tb;
-  if (!encode_kmajor_map(&ta, hidden, rows, H, kBM) || !encode_kmajor_map(&tb, w_lm, V, H, kBN))
-    return TV_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned long long* keys = static_cast<unsigned long long*>(workspace);
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Tile width: 256 columns, unless the grid is a few waves of one CTA per SM
+  // (few rows: the weights stream at the SMs' pull rate); then the multiple of
+  // 32 in [128, 256] with the fewest waves x columns, so that the last wave is
+  // not left mostly empty (V = 32000: 125 tiles of 256 leave 23 of 148 SMs
+  // idle, 143 tiles of 224 leave 5).
+  int bn = kBN;
+  if ((int64_t)m_tiles * (((int64_t)V + kBN - 1) / kBN) <= 8LL * sms) {
+    int64_t best = -1;
+    for (int cand = kBN; cand >= 128; cand -= 32) {
+      const int64_t tiles = (int64_t)m_tiles * (((int64_t)V + cand - 1) / cand);
+      const int64_t cost = (tiles + sms - 1) / sms * cand;
+      if (best < 0 || cost < best) {
+        best = cost;
+        bn = cand;
+      }
+    }
+  }
+  const int64_t n_tiles = ((int64_t)V + bn - 1) / bn;
+  if ((int64_t)m_tiles * n_tiles > 0x7fffffffLL) return TV_ERR_UNSUPPORTED;
+  CUtensorMap ta, tb;
+  if (!encode_kmajor_map(&ta, hidden, rows, H, kBM) || !encode_kmajor_map(&tb, w_lm, V, H, bn))
+    return TV_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned long long* keys = static_cast<unsigned long long*>(workspace);
   const unsigned small_grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((rows + 255) / 256, sms));
   tv_status r = launch(lm_keys_init_kernel, dim3(small_grid), dim3(kLmThreads), 0, s, 1, true, keys, rows);
   if (r != TV_OK) return r;
@@ -261,7 +280,7 @@ extern "C" tv_status tree_accept_lm_head(const uint16_t* hidden, const uint16_t*
   e = cudaFuncSetAttribute(lm_head_argmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return record_cuda_error(e);
   r = launch(lm_head_argmax_kernel, dim3((unsigned)(m_tiles * n_tiles)), dim3(kLmThreads), smem, s, 1, true, ta, tb,
-             (int)rows, H, V, m_tiles, M + 1, keys, status, pipeline_wait_limit_ns());
+             (int)rows, H, V, m_tiles, bn, M + 1, keys, status, pipeline_wait_limit_ns());
   if (r != TV_OK) return r;
   r = launch(lm_keys_decode_kernel, dim3(small_grid), dim3(256), 0, s, 1, true, (const unsigned long long*)keys,
              argmax, rows);
