@@ -14,14 +14,16 @@
 // each CTA's shared memory and merging over distributed shared memory gave the
 // same bits and measured no faster on B200.)
 // Warp roles (192 threads):
-//   warp 0      TMA producer: 64-key K tiles and V tiles into two separate smem
-//               rings -- a K slot is freed as soon as S = QK^T has read it, a V
-//               slot only after O += PV, so the V ring is the deeper one
+//   warp 0      TMA producer: lane 0 streams 64-key K tiles and lane 1 V tiles
+//               into two separate smem rings (two slots each with two CTAs per
+//               SM) -- a K slot is freed once S = QK^T has read it, a V slot
+//               after O += PV
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_i = Q K_i^T   (M=128, N=64, K=128; A, B from smem)   -> TMEM S[i%2]
 //                 O  += P_i V_i   (M=128, N=128, K=64; A=P from TMEM, B=V from smem) -> TMEM O
-//               S_{i+1} is issued before waiting for P_i, so the tensor core
-//               computes the next scores while the softmax warps work.
+//               it polls its K, P and V barriers and issues whichever MMA is
+//               ready, so S_{i+1} is computed while the softmax warps work on
+//               S_i, and a late K tile holds back no PV (nor a late V tile a QK)
 //   warps 2-5   softmax: thread t owns TMEM lane t, i.e. query row t; it reads
 //               its 64 scores with one tcgen05.ld, keeps the running max / sum,
 //               writes P (bf16) over its scores, and rescales its O row only
