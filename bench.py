@@ -71,7 +71,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU work budget of each oracle baseline sample (one thread and all cores)")
-    ap.add_argument("--layers", type=int, default=0, help="cap on the distinct layer buffers (profiling runs)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="cap on the distinct layer buffers; with --profile commit, the layers committed")
     ap.add_argument("--rounds", type=int, default=0, help="rounds of a multi-round workload (0: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
@@ -1258,7 +1259,9 @@ def run_profile(args, cfg):
     device = torch.device("cuda", 0)
     if args.batch:
         cfg = dataclasses.replace(cfg, B=args.batch)
-    cfg = dataclasses.replace(cfg, L=1)
+    # one layer, or with --layers that many for the commit (its launch moves
+    # every layer's rows: a few layers keep the moved bytes above L2)
+    cfg = dataclasses.replace(cfg, L=args.layers if (args.profile == "commit" and args.layers > 0) else 1)
     stream = torch.cuda.current_stream(device)
     if args.profile == "lm_head":
         H = cfg.Hq * cfg.D
